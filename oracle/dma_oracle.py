@@ -1,0 +1,378 @@
+"""Plain CPU oracle for the Dynamic Mask Attention (DMA) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA library and never calls it; it is deliberately slow and written to be
+checked by eye against the method's definition on the page "Trainable Dynamic
+Mask Sparse Attention: Bridging Efficiency and Effectiveness in Long-Context
+Language Models" (Hugging Face blog "dmattn"):
+
+  * gate      -- section "Dynamic Sparse Mask Generation", equation for delta
+                 ("Dynamic Weight Computation"): delta = exp(tau(v Delta) x A);
+  * selection -- same section, equation for m_t ("Mask Combination with Causal
+                 Constraints"): m_t = f(top_w(delta + m_c^t));
+  * attention -- section "Efficient Sparse Attention Computation", equation for
+                 o_t: o_t = softmax(q_t k^T / sqrt(d_h) (+) m_t) v;
+  * backward  -- "Theoretical Guarantees for Safe Computation Skipping" (masked
+                 pairs give exactly zero weight and zero gradient) and
+                 "Gradient Flow Integrity" (end-to-end trainable).
+
+Readings where the page is silent or garbled (each repeated where it is used):
+  tau = softplus; v at key position j is the concatenation of the Hkv key/value
+  heads (length Hkv*d), Delta is [Hkv*d, H], and delta is per query head;
+  the mask is ADDED to the scaled scores (selected key j contributes
+  +delta_j, others -inf); top-w orders keys by delta descending and breaks ties
+  toward the lower key index; a row with fewer than w causal keys keeps all of
+  them; the selection is a constant in the backward pass; LSE is the natural
+  log of the softmax denominator.
+
+Precision: float64 throughout unless a caller asks for float32 GEMMs on large
+inputs (reductions stay in float64).
+
+Parity pins: see tests/test_oracle_*.py.  Every function below is pinned by a
+test that does not re-type its formula (brute force, closed forms, library
+routines on special cases, finite differences, invariants).
+"""
+from __future__ import annotations
+
+import heapq
+import math
+
+import numpy as np
+
+__all__ = [
+    "softplus",
+    "sigmoid",
+    "gate",
+    "topw_sets_bruteforce",
+    "topw_eviction",
+    "mask_from_eviction",
+    "eviction_from_mask",
+    "live_keys_per_block",
+    "attn_fwd",
+    "attn_bwd",
+    "gate_bwd",
+    "decode_select",
+    "decode_attn",
+]
+
+
+# ----------------------------------------------------------------------------
+# Gate: delta = exp(tau(v Delta) * A), tau = softplus
+# ----------------------------------------------------------------------------
+
+def softplus(x: np.ndarray) -> np.ndarray:
+    """tau(x) = ln(1 + e^x), the non-negative function of the delta equation
+    (reading: softplus).  Written in the overflow-free form
+    max(x, 0) + ln(1 + e^{-|x|})."""
+    x = np.asarray(x, dtype=np.float64)
+    return np.maximum(x, 0.0) + np.log1p(np.exp(-np.abs(x)))
+
+
+def sigmoid(x: np.ndarray) -> np.ndarray:
+    """Derivative of softplus, 1 / (1 + e^{-x}), evaluated without overflow."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    pos = x >= 0
+    out[pos] = 1.0 / (1.0 + np.exp(-x[pos]))
+    ex = np.exp(x[~pos])
+    out[~pos] = ex / (1.0 + ex)
+    return out
+
+
+def gate(V: np.ndarray, Delta: np.ndarray, A: np.ndarray, gemm_dtype=np.float64):
+    """Content-aware gate ("Dynamic Weight Computation" equation).
+
+    V      [B, Hkv, N, d]  value vectors.
+    Delta  [Hkv*d, H]      learnable sampling weights.
+    A      [H]             per-head selective control.
+
+    Reading: the value vector of key position j is the concatenation over the
+    Hkv heads, v_j[g*d + c] = V[b, g, j, c]; x = v Delta is [B, N, H];
+    delta = exp(A_h * softplus(x)) is one value per (batch, query head, key).
+
+    Returns (x, delta), both [B, H, N] float64.
+    """
+    B, Hkv, N, d = V.shape
+    H = Delta.shape[1]
+    assert Delta.shape == (Hkv * d, H)
+    v = np.asarray(V, dtype=gemm_dtype).transpose(0, 2, 1, 3).reshape(B, N, Hkv * d)
+    x = np.matmul(v, np.asarray(Delta, dtype=gemm_dtype)).astype(np.float64)  # [B, N, H]
+    x = x.transpose(0, 2, 1).copy()  # [B, H, N]
+    delta = np.exp(np.asarray(A, dtype=np.float64)[None, :, None] * softplus(x))
+    return x, delta
+
+
+# ----------------------------------------------------------------------------
+# Causal top-w selection: m_t = f(top_w(delta + m_c^t))
+# ----------------------------------------------------------------------------
+
+def _better(di: float, i: int, dj: float, j: int) -> bool:
+    """Total order of the top-w selection: larger delta first; equal delta ->
+    lower key index first (tie reading)."""
+    return di > dj or (di == dj and i < j)
+
+
+def topw_sets_bruteforce(delta_row: np.ndarray, w: int) -> np.ndarray:
+    """Selection by the definition, one query at a time.
+
+    For query t the causal constraint m_c^t removes keys j > t; top_w keeps
+    the min(t+1, w) best of the remaining keys; f sends every other key to
+    -inf.  Returns the boolean mask M[t, j] (True = selected).  O(N^2 log N):
+    for tiny inputs only.
+    """
+    d = [float(v) for v in np.asarray(delta_row, dtype=np.float32)]
+    N = len(d)
+    M = np.zeros((N, N), dtype=bool)
+    for t in range(N):
+        order = sorted(range(t + 1), key=lambda j: (-d[j], j))
+        for j in order[: min(t + 1, w)]:
+            M[t, j] = True
+    return M
+
+
+def topw_eviction(delta_row: np.ndarray, w: int) -> np.ndarray:
+    """Eviction index of every key, from one sequential pass.
+
+    Because delta depends on the key but not on the query, the rank of key j
+    among keys 0..t can only grow with t, so key j is selected exactly for the
+    queries t in [j, e_j).  The pass keeps the current selection in a min-heap
+    ordered by the selection order; after key t is pushed the worst member is
+    popped whenever the heap holds more than w keys, and that key's e is t.
+    Keys never popped get e = N.  e_j == j means key j is never selected.
+    """
+    d = np.asarray(delta_row, dtype=np.float32)
+    N = d.shape[0]
+    e = np.full(N, N, dtype=np.int64)
+    heap: list[tuple[float, int]] = []   # (delta, -j): smallest = worst
+    for t in range(N):
+        heapq.heappush(heap, (float(d[t]), -t))
+        if len(heap) > w:
+            _, negj = heapq.heappop(heap)
+            e[-negj] = t
+    return e
+
+
+def mask_from_eviction(e: np.ndarray, q_rows: np.ndarray | None = None) -> np.ndarray:
+    """M[t, j] = (j <= t < e_j) for the query rows q_rows (default 0..N-1)."""
+    N = e.shape[-1]
+    t = np.arange(N) if q_rows is None else np.asarray(q_rows)
+    j = np.arange(N)
+    return (j[None, :] <= t[:, None]) & (t[:, None] < e[None, :])
+
+
+def eviction_from_mask(M: np.ndarray) -> np.ndarray:
+    """Inverse of mask_from_eviction for a full [N, N] mask that has the
+    interval form; raises if some key's selected queries are not an interval
+    starting at the key itself."""
+    N = M.shape[0]
+    e = np.empty(N, dtype=np.int64)
+    for j in range(N):
+        col = M[:, j]
+        ts = np.nonzero(col)[0]
+        if ts.size == 0:
+            e[j] = j
+            continue
+        if ts[0] != j or ts[-1] - ts[0] + 1 != ts.size:
+            raise ValueError(f"key {j}: selected queries are not an interval from j")
+        e[j] = ts[-1] + 1
+    return e
+
+
+def live_keys_per_block(e: np.ndarray, Bq: int):
+    """Keys a query block [t0, t0+Bq) attends to, split into 'full' keys
+    (selected by every query row of the block) and 'partial' keys.
+
+    Returns a list over blocks of (full: sorted int array, partial: sorted int
+    array).  A key is full when j <= t0 and e_j >= t0 + Bq (so in a ragged
+    last block, where rows past N do not exist, surviving keys still count as
+    partial: they are masked, which is always correct).
+    """
+    N = e.shape[0]
+    j = np.arange(N)
+    out = []
+    for t0 in range(0, N, Bq):
+        t1 = min(t0 + Bq, N)
+        live = (j < t1) & (e > np.maximum(j, t0))
+        full = live & (j <= t0) & (e >= t0 + Bq)
+        out.append((np.nonzero(full)[0], np.nonzero(live & ~full)[0]))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Masked attention forward / backward
+# ----------------------------------------------------------------------------
+
+def _scores(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype):
+    """Scaled scores plus the additive mask of rows `rows`.
+
+    Reading of the garbled operator in the o_t equation: the mask m_t is added
+    to q_t k^T / sqrt(d): selected key j contributes +delta_j, non-selected
+    keys -inf (f of the m_t equation)."""
+    N = Kg.shape[0]
+    s = np.matmul(np.asarray(Qh[rows], dtype=gemm_dtype),
+                  np.asarray(Kg, dtype=gemm_dtype).T).astype(np.float64) * scale
+    s = s + np.asarray(delta_h, dtype=np.float64)[None, :]
+    t = np.asarray(rows)[:, None] if rows is not None else np.arange(Qh.shape[0])[:, None]
+    j = np.arange(N)[None, :]
+    sel = (j <= t) & (t < np.asarray(e_h)[None, :])
+    return np.where(sel, s, -np.inf), sel
+
+
+def attn_fwd(Q, K, V, delta, evict, scale=None, q_pos0: int = 0, rows=None,
+             gemm_dtype=np.float64, chunk: int = 1024):
+    """Masked attention forward ("Efficient Sparse Attention Computation").
+
+    Q [B, H, Nq, d] (query row i sits at position q_pos0 + i), K, V
+    [B, Hkv, N, d], delta [B, H, N], evict [B, H, N] (the selection as
+    eviction indices).  Returns O [B, H, Nq, d] and LSE [B, H, Nq] (natural log
+    of the softmax denominator), float64.  `rows` restricts the computation to
+    a subset of query rows (other rows are NaN).
+
+    Dense definition: every causal key is scored, non-selected ones get -inf,
+    softmax with max subtraction, O = P V.
+    """
+    if q_pos0 != 0:
+        raise NotImplementedError("query rows at an offset: use decode_attn")
+    B, H, Nq, d = Q.shape
+    Hkv, N = K.shape[1], K.shape[2]
+    G = H // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    O = np.full((B, H, Nq, d), np.nan)
+    LSE = np.full((B, H, Nq), np.nan)
+    all_rows = np.arange(Nq) if rows is None else np.asarray(rows)
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            for c0 in range(0, all_rows.size, chunk):
+                r = all_rows[c0:c0 + chunk]
+                s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], r, scale, gemm_dtype)
+                m = s.max(axis=1, keepdims=True)
+                p = np.exp(s - m)
+                l = p.sum(axis=1, keepdims=True)
+                O[b, h, r] = np.matmul(p / l, np.asarray(V[b, g], dtype=gemm_dtype)).astype(np.float64)
+                LSE[b, h, r] = (m + np.log(l))[:, 0]
+    return O, LSE
+
+
+def attn_bwd(Q, K, V, delta, evict, dO, scale=None, gemm_dtype=np.float64):
+    """Analytic backward of attn_fwd with the selection held constant.
+
+    With P the masked softmax and L = sum(dO * O):
+      dP = dO V^T,  D_t = sum_c dO_tc O_tc = sum_j P_tj dP_tj,
+      dS = P * (dP - D),
+      dQ = scale * dS K,   dK_g = scale * sum_{h in g} dS_h^T Q_h,
+      dV_g = sum_{h in g} P_h^T dO_h,   ddelta_h = column sums of dS_h.
+    Masked pairs have P = 0 hence dS = 0: zero gradient, as the section
+    "Theoretical Guarantees for Safe Computation Skipping" states.
+
+    Returns dQ [B,H,N,d], dK, dV [B,Hkv,N,d], ddelta [B,H,N], all float64.
+    """
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    G = H // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dQ = np.zeros((B, H, N, d))
+    dK = np.zeros((B, Hkv, N, d))
+    dV = np.zeros((B, Hkv, N, d))
+    ddelta = np.zeros((B, H, N))
+    rows = np.arange(N)
+    f = lambda a: np.asarray(a, dtype=gemm_dtype)
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], rows, scale, gemm_dtype)
+            m = s.max(axis=1, keepdims=True)
+            p = np.exp(s - m)
+            P = p / p.sum(axis=1, keepdims=True)
+            dP = np.matmul(f(dO[b, h]), f(V[b, g]).T).astype(np.float64)
+            Dt = (P * dP).sum(axis=1, keepdims=True)
+            dS = P * (dP - Dt)
+            dQ[b, h] = scale * np.matmul(f(dS), f(K[b, g])).astype(np.float64)
+            dK[b, g] += scale * np.matmul(f(dS).T, f(Q[b, h])).astype(np.float64)
+            dV[b, g] += np.matmul(f(P).T, f(dO[b, h])).astype(np.float64)
+            ddelta[b, h] = dS.sum(axis=0)
+    return dQ, dK, dV, ddelta
+
+
+# ----------------------------------------------------------------------------
+# Gate backward (Delta and A are learnable; the method is end-to-end trainable)
+# ----------------------------------------------------------------------------
+
+def gate_bwd(V, Delta, A, ddelta, gemm_dtype=np.float64):
+    """Gradients of sum(ddelta * delta) with delta = exp(A * softplus(v Delta)).
+
+    d delta / d x = delta * A * sigmoid(x),  d delta / d A = delta * softplus(x).
+    With gx = ddelta * delta * A * sigmoid(x):
+      dA_h        = sum_{b,j} ddelta * delta * softplus(x),
+      dDelta[r,h] = sum_{b,j} v_j[r] * gx[b,h,j],
+      dV_gate[b,g,j,c] = sum_h gx[b,h,j] * Delta[g*d+c, h].
+    The gate's share of dV is returned on its own (the caller adds it to the
+    attention's dV).  Returns (dDelta [Hkv*d,H], dA [H], dV_gate [B,Hkv,N,d]).
+    """
+    B, Hkv, N, d = V.shape
+    H = Delta.shape[1]
+    x, delta = gate(V, Delta, A, gemm_dtype=gemm_dtype)
+    dd = np.asarray(ddelta, dtype=np.float64)
+    A64 = np.asarray(A, dtype=np.float64)
+    gx = dd * delta * A64[None, :, None] * sigmoid(x)          # [B, H, N]
+    dA = (dd * delta * softplus(x)).sum(axis=(0, 2))           # [H]
+    v = np.asarray(V, dtype=np.float64).transpose(0, 2, 1, 3).reshape(B, N, Hkv * d)
+    dDelta = np.einsum("bnr,bhn->rh", v, gx)
+    dvf = np.einsum("bhn,rh->bnr", gx, np.asarray(Delta, dtype=np.float64))   # [B, N, Hkv*d]
+    dV_gate = dvf.reshape(B, N, Hkv, d).transpose(0, 2, 1, 3).copy()
+    return dDelta, dA, dV_gate
+
+
+# ----------------------------------------------------------------------------
+# Decode: one new query at position L-1 over an L-row cache
+# ----------------------------------------------------------------------------
+
+def decode_select(delta: np.ndarray, w: int) -> np.ndarray:
+    """Keys selected for a query at position L-1 (all L keys are causal):
+    the min(L, w) best under the selection order (delta descending, lower
+    index first on ties).  Returns int64 [B, H, min(L, w)] sorted ascending by
+    key index (the "Unified Training-Inference Architecture" section: the same
+    selection at inference)."""
+    B, H, L = delta.shape
+    k = min(L, w)
+    out = np.empty((B, H, k), dtype=np.int64)
+    idx = np.arange(L)
+    for b in range(B):
+        for h in range(H):
+            d = np.asarray(delta[b, h], dtype=np.float32).astype(np.float64)
+            order = np.lexsort((idx, -d))       # primary -delta, secondary index
+            out[b, h] = np.sort(order[:k])
+    return out
+
+
+def decode_attn(q, K, V, delta, sel, scale=None):
+    """o = softmax(q k_j^T * scale + delta_j over the selected j) V.
+
+    q [B, H, d] (or [B, H, 1, d]), K, V [B, Hkv, L, d], delta [B, H, L],
+    sel [B, H, k] selected key indices.  Returns o [B, H, d], lse [B, H]."""
+    q = np.asarray(q)
+    if q.ndim == 4:
+        q = q[:, :, 0, :]
+    B, H, d = q.shape
+    Hkv = K.shape[1]
+    G = H // Hkv
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = np.empty((B, H, d))
+    lse = np.empty((B, H))
+    for b in range(B):
+        for h in range(H):
+            g = h // G
+            j = sel[b, h]
+            kk = np.asarray(K[b, g, j], dtype=np.float64)
+            vv = np.asarray(V[b, g, j], dtype=np.float64)
+            s = kk @ np.asarray(q[b, h], dtype=np.float64) * scale + np.asarray(delta[b, h, j], dtype=np.float64)
+            m = s.max()
+            p = np.exp(s - m)
+            l = p.sum()
+            o[b, h] = (p / l) @ vv
+            lse[b, h] = m + math.log(l)
+    return o, lse
