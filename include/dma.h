@@ -1,0 +1,213 @@
+/*
+ * dma.h -- C ABI of the Dynamic Mask Attention (DMA) hot path for NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described on the page "Trainable Dynamic Mask Sparse Attention:
+ * Bridging Efficiency and Effectiveness in Long-Context Language Models" (Hugging Face blog
+ * "dmattn", arXiv 2508.02124).  Three steps run on the GPU:
+ *
+ *   1. gate       delta = exp(softplus(v Delta) * A)           (section "Dynamic Sparse Mask
+ *                                                              Generation", delta equation)
+ *   2. mask       m_t = f(top_w(delta + m_c^t))                (same section, m_t equation)
+ *   3. attention  o_t = softmax(q_t k^T / sqrt(d) + m_t) v     (section "Efficient Sparse
+ *                                                              Attention Computation", o_t
+ *                                                              equation), forward and backward
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every call is asynchronous on the caller's CUDA stream (`stream` is a cudaStream_t passed
+ *    as void*; NULL is the legacy default stream).  No call synchronises the host, allocates
+ *    device memory, or keeps a pointer after its stream work completes.  The library has no
+ *    mutable global state; calls on different streams may run concurrently when their buffers
+ *    (including workspaces) are distinct.
+ *  - All pointers are device pointers, 16-byte aligned, to dense row-major (C-contiguous)
+ *    tensors with the layouts given per argument.  The caller owns every buffer.
+ *  - Arguments are validated before anything is launched.  On any error nothing is launched
+ *    and no output is touched, except DMA_ERR_CUDA, which reports a failed launch (outputs are
+ *    then unspecified).
+ *  - Outputs are fully overwritten, never accumulated into.
+ *  - Tensor names follow the page: Q, K, V, Delta (the sampling weights), A (per-head
+ *    selective control), delta (the dynamic weights), O, LSE.
+ *
+ * Readings of points the page leaves open (also listed in the project design notes):
+ *  - tau is softplus.  The value vector of key position j is the concatenation of its Hkv
+ *    value heads (length Hkv*d); Delta is [Hkv*d, H]; delta has one value per query head.
+ *  - The mask is ADDED to the scaled scores: a selected key j contributes +delta_j, any
+ *    other key -inf.  The scale multiplies q k^T only.
+ *  - top-w orders keys by delta descending and breaks ties toward the lower key index
+ *    (-0.0 compares equal to +0.0).  A query at position t with t+1 <= w keeps all of its
+ *    causal keys; the query's own key competes like any other.  NaN gate values are not
+ *    supported (their selection is unspecified).
+ *  - In the backward pass the selection is a constant: gradients reach delta only through
+ *    the additive bias of selected pairs.  Masked pairs get exactly zero gradient (section
+ *    "Theoretical Guarantees for Safe Computation Skipping").
+ *  - LSE is the natural logarithm of the softmax denominator sum_j exp(s_tj).
+ */
+#ifndef DMA_H_
+#define DMA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DMA_ABI_VERSION 1
+
+/* Query rows per block of the mask encoding and of the attention kernels. */
+#define DMA_BLOCK_Q 128
+
+typedef enum {
+  DMA_OK = 0,
+  DMA_ERR_INVALID_ARG = 1, /* a NULL/misaligned pointer, an inconsistent or out-of-range size */
+  DMA_ERR_UNSUPPORTED = 2, /* a valid request outside what the kernels implement (see limits) */
+  DMA_ERR_WORKSPACE = 3,   /* workspace NULL or smaller than dma_workspace_size() */
+  DMA_ERR_CUDA = 4,        /* a CUDA launch failed (cudaGetLastError after the launch) */
+  DMA_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up (see dma_check_device_status) */
+} dma_status_t;
+
+typedef enum {
+  DMA_BF16 = 0, /* Q, K, V, Delta, dO, O, dQ, dK, dV stored as bfloat16 */
+  DMA_F32 = 1   /* stored as float32 (the gate then runs on float32 values; the attention
+                   kernels round Q, K, V to bfloat16 in their load stage) */
+} dma_dtype_t;
+
+/*
+ * Problem description.
+ *   B      batch
+ *   H      query heads;  Hkv key/value heads, H % Hkv == 0 (grouped-query attention:
+ *          query head h reads key/value head h / (H / Hkv))
+ *   N      key length (sequence length, or cache length for decode)
+ *   Nq     query rows: Nq == N (prefill / training; query row i sits at position i) or
+ *          Nq == 1 (decode; the single query sits at position N-1)
+ *   d      head dimension, 64 or 128
+ *   w      window of the top-w selection, w >= 1 (w >= N keeps every causal key)
+ *   scale  multiplier of q k^T; a value <= 0 selects 1/sqrt(d)
+ *   dtype  a dma_dtype_t
+ *
+ * Limits of this implementation (DMA_ERR_UNSUPPORTED beyond them): prefill/training
+ * N <= 16384; decode N <= 1<<24; B*H <= 65535; d in {64, 128}.
+ */
+typedef struct {
+  int32_t B, H, Hkv, N, Nq, d, w;
+  float scale;
+  int32_t dtype;
+} dma_params_t;
+
+/*
+ * Workspace layout.  The workspace is one caller-allocated device buffer of at least
+ * dma_workspace_size() bytes, passed to every call of one problem.  Its leading regions are
+ * part of the ABI so that callers and tests can read the mask encoding:
+ *
+ *   off_status  int32 device status word (0 = ok), written by bounded waits.
+ *   off_counts  int32 [B, H, n_blocks, 2]: per query block, (n_full, n_live).
+ *   off_lists   int32 [B, H, n_blocks, list_cap]: the live keys of each query block, the
+ *               n_full "full" keys (selected by every row of the block) first, then the
+ *               partial ones; each group in ascending key order.  Entries past n_live are
+ *               unspecified.
+ *   off_sel     decode only: int32 [B, H, sel_len] selected keys of the query, ascending.
+ *   the rest    internal scratch.
+ */
+typedef struct {
+  size_t bytes;
+  size_t off_status;
+  size_t off_counts;
+  size_t off_lists;
+  size_t off_sel;
+  int32_t n_blocks;
+  int32_t list_cap;
+  int32_t sel_len;
+  int32_t reserved;
+} dma_ws_layout_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* dma_status_string(dma_status_t status);
+
+/* DMA_ABI_VERSION of the loaded library. */
+int32_t dma_abi_version(void);
+
+/* Bytes of workspace every call of problem `p` needs (covers all entry points). */
+dma_status_t dma_workspace_size(const dma_params_t* p, size_t* bytes);
+
+/* Offsets of the ABI-visible workspace regions for problem `p`. */
+dma_status_t dma_workspace_layout(const dma_params_t* p, dma_ws_layout_t* layout);
+
+/*
+ * Gate (delta equation).
+ *   V       [B, Hkv, N, d]   dtype
+ *   Delta   [Hkv*d, H]       dtype
+ *   A       [H]              float32
+ *   delta   [B, H, N]        float32 out: exp(A_h * softplus(x)),  x[b,h,j] = sum_r v_j[r] Delta[r,h]
+ *   x_save  [B, H, N]        float32 out, may be NULL: x, kept for dma_gate_bwd
+ * x is accumulated in float32 (bf16 products are exact in float32).
+ */
+dma_status_t dma_gate(const dma_params_t* p, const void* V, const void* Delta, const float* A,
+                      float* delta, float* x_save, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * Causal top-w mask (m_t equation), encoded exactly.
+ *   delta  [B, H, N] float32 in
+ *   evict  [B, H, N] int32 out (prefill/training): e_j = the first query position at which key
+ *          j is no longer among the w best causal keys (N if never).  Query t selects key j
+ *          iff j <= t < e_j; e_j == j means key j is never selected.  Because delta does not
+ *          depend on the query, the queries selecting a key always form this interval.
+ *          Also writes the per-block live-key lists and counts into the workspace.
+ *          Decode (Nq == 1): `evict` must be NULL; the selected keys of the query at
+ *          position N-1 are written to the workspace region off_sel.
+ */
+dma_status_t dma_topk_mask(const dma_params_t* p, const float* delta, int32_t* evict,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Masked attention forward (o_t equation), computing only on the live keys of each block
+ * (masked pairs are skipped, section "Theoretical Guarantees for Safe Computation Skipping").
+ *   Q      [B, H, Nq, d] dtype;  K, V [B, Hkv, N, d] dtype;  delta [B, H, N] float32
+ *   evict  [B, H, N] int32 from dma_topk_mask (NULL for decode); the workspace must hold the
+ *          lists (or selection) dma_topk_mask wrote for the same delta.
+ *   O      [B, H, Nq, d] dtype out;  LSE [B, H, Nq] float32 out
+ */
+dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
+                          const float* delta, const int32_t* evict, void* workspace,
+                          size_t workspace_bytes, void* O, float* LSE, void* stream);
+
+/*
+ * Masked attention backward (prefill/training only), selection held constant.
+ *   O, LSE from dma_attn_fwd; dO [B, H, N, d] dtype.
+ *   dQ [B, H, N, d], dK, dV [B, Hkv, N, d] dtype out (dK, dV summed over the query heads of
+ *   each group);  d_delta [B, H, N] float32 out (sum over queries of dS_tj).
+ */
+dma_status_t dma_attn_bwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
+                          const float* delta, const int32_t* evict, void* workspace,
+                          size_t workspace_bytes, const void* O, const float* LSE,
+                          const void* dO, void* dQ, void* dK, void* dV, float* d_delta,
+                          void* stream);
+
+/*
+ * Gate backward (Delta and A are learnable; the method is trainable end to end, section
+ * "Gradient Flow Integrity").  With gx = d_delta * delta * A * sigmoid(x):
+ *   dDelta  [Hkv*d, H] float32 out:  sum_{b,j} v_j[r] gx[b,h,j]
+ *   dA      [H] float32 out:         sum_{b,j} d_delta * delta * softplus(x)
+ *   dV_gate [B, Hkv, N, d] float32 out: sum_h gx[b,h,j] Delta[g*d+c, h]  (the gate's share of
+ *           dV; the caller adds it to dma_attn_bwd's dV)
+ *   x_save, delta: from dma_gate on the same V, Delta, A (x_save must not be NULL).
+ */
+dma_status_t dma_gate_bwd(const dma_params_t* p, const void* V, const void* Delta,
+                          const float* A, const float* x_save, const float* delta,
+                          const float* d_delta, float* dDelta, float* dA, float* dV_gate,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads the device status word of `workspace` (synchronises `stream`).  Returns DMA_OK or
+ * DMA_ERR_TIMEOUT when a kernel's bounded wait gave up; *code receives the raw word.
+ * dma_clear_device_status resets it (asynchronously on `stream`).
+ */
+dma_status_t dma_check_device_status(const dma_params_t* p, void* workspace, void* stream,
+                                     int32_t* code);
+dma_status_t dma_clear_device_status(const dma_params_t* p, void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMA_H_ */

@@ -256,7 +256,7 @@ def attn_fwd(Q, K, V, delta, evict, scale=None, q_pos0: int = 0, rows=None,
     return O, LSE
 
 
-def attn_bwd(Q, K, V, delta, evict, dO, scale=None, gemm_dtype=np.float64):
+def attn_bwd(Q, K, V, delta, evict, dO, scale=None, gemm_dtype=np.float64, chunk: int = 1024):
     """Analytic backward of attn_fwd with the selection held constant.
 
     With P the masked softmax and L = sum(dO * O):
@@ -266,6 +266,8 @@ def attn_bwd(Q, K, V, delta, evict, dO, scale=None, gemm_dtype=np.float64):
       dV_g = sum_{h in g} P_h^T dO_h,   ddelta_h = column sums of dS_h.
     Masked pairs have P = 0 hence dS = 0: zero gradient, as the section
     "Theoretical Guarantees for Safe Computation Skipping" states.
+    Query rows are processed `chunk` at a time (sums over rows accumulate
+    across chunks) so that large inputs fit in memory.
 
     Returns dQ [B,H,N,d], dK, dV [B,Hkv,N,d], ddelta [B,H,N], all float64.
     """
@@ -278,22 +280,24 @@ def attn_bwd(Q, K, V, delta, evict, dO, scale=None, gemm_dtype=np.float64):
     dK = np.zeros((B, Hkv, N, d))
     dV = np.zeros((B, Hkv, N, d))
     ddelta = np.zeros((B, H, N))
-    rows = np.arange(N)
     f = lambda a: np.asarray(a, dtype=gemm_dtype)
     for b in range(B):
         for h in range(H):
             g = h // G
-            s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], rows, scale, gemm_dtype)
-            m = s.max(axis=1, keepdims=True)
-            p = np.exp(s - m)
-            P = p / p.sum(axis=1, keepdims=True)
-            dP = np.matmul(f(dO[b, h]), f(V[b, g]).T).astype(np.float64)
-            Dt = (P * dP).sum(axis=1, keepdims=True)
-            dS = P * (dP - Dt)
-            dQ[b, h] = scale * np.matmul(f(dS), f(K[b, g])).astype(np.float64)
-            dK[b, g] += scale * np.matmul(f(dS).T, f(Q[b, h])).astype(np.float64)
-            dV[b, g] += np.matmul(f(P).T, f(dO[b, h])).astype(np.float64)
-            ddelta[b, h] = dS.sum(axis=0)
+            Kg, Vg = f(K[b, g]), f(V[b, g])
+            for c0 in range(0, N, chunk):
+                rows = np.arange(c0, min(N, c0 + chunk))
+                s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], rows, scale, gemm_dtype)
+                m = s.max(axis=1, keepdims=True)
+                p = np.exp(s - m)
+                P = p / p.sum(axis=1, keepdims=True)
+                dP = np.matmul(f(dO[b, h, rows]), Vg.T).astype(np.float64)
+                Dt = (P * dP).sum(axis=1, keepdims=True)
+                dS = P * (dP - Dt)
+                dQ[b, h, rows] = scale * np.matmul(f(dS), Kg).astype(np.float64)
+                dK[b, g] += scale * np.matmul(f(dS).T, f(Q[b, h, rows])).astype(np.float64)
+                dV[b, g] += np.matmul(f(P).T, f(dO[b, h, rows])).astype(np.float64)
+                ddelta[b, h] += dS.sum(axis=0)
     return dQ, dK, dV, ddelta
 
 

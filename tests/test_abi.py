@@ -1,0 +1,155 @@
+"""The C-ABI library loads, exports every entry point include/dma.h declares,
+and validates arguments on the host before launching anything.  No test here
+touches a GPU: every call below is rejected by host-side checks."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import trainable_dynamic_mask_b200 as dma
+from trainable_dynamic_mask_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dma.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from trainable_dynamic_mask_b200 import build
+        build.build()
+    return dma.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dma_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    names = declared_functions()
+    assert len(names) >= 11
+    lib = dma.load()
+    for n in names:
+        assert hasattr(lib, n), f"{n} missing from libdma.so"
+    assert sorted(_lib.exported_names()) == names
+
+
+def test_abi_version_and_status_strings():
+    assert dma.abi_version() == 1
+    lib = dma.load()
+    for code in range(6):
+        s = lib.dma_status_string(code).decode()
+        assert s.startswith(_lib.STATUS_NAMES[code])
+    assert lib.dma_status_string(99).decode() == "DMA_ERR_UNKNOWN"
+
+
+def _ws_size(p):
+    n = ctypes.c_size_t(0)
+    st = dma.load().dma_workspace_size(ctypes.byref(p), ctypes.byref(n))
+    return st, n.value
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=64), OK),
+    (dict(B=1, H=3, Hkv=2, N=256, d=64, w=64), INVALID),        # H % Hkv
+    (dict(B=1, H=2, Hkv=1, N=256, d=96, w=64), UNSUPPORTED),    # head dim
+    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=0), INVALID),         # window
+    (dict(B=0, H=2, Hkv=1, N=256, d=64, w=4), INVALID),
+    (dict(B=1, H=2, Hkv=1, N=16385, d=64, w=4), UNSUPPORTED),   # prefill row limit
+    (dict(B=1, H=2, Hkv=1, N=16384, d=128, w=4), OK),
+    (dict(B=1, H=2, Hkv=1, N=65536, d=128, w=4, Nq=1), OK),     # decode has no such limit
+    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=4, Nq=7), INVALID),   # Nq must be N or 1
+    (dict(B=300, H=256, Hkv=1, N=256, d=64, w=4), UNSUPPORTED), # grid limit on B*H
+])
+def test_params_validation(kw, expect):
+    p = dma.make_params(**kw)
+    st, _ = _ws_size(p)
+    assert st == expect
+
+
+def test_bad_dtype_and_scale():
+    p = dma.make_params(1, 2, 1, 256, 64, 64)
+    p.dtype = 7
+    assert _ws_size(p)[0] == INVALID
+    p = dma.make_params(1, 2, 1, 256, 64, 64, scale=float("nan"))
+    assert _ws_size(p)[0] == INVALID
+
+
+def test_workspace_layout_plan():
+    p = dma.make_params(B=1, H=16, Hkv=8, N=4096, d=128, w=1024)
+    lay = dma.workspace_layout(p)
+    assert lay.n_blocks == 32
+    assert lay.list_cap == 1024 + 128
+    assert lay.sel_len == 0
+    for off in (lay.off_status, lay.off_counts, lay.off_lists):
+        assert off % 256 == 0
+    assert lay.off_counts >= lay.off_status + 4
+    assert lay.off_lists >= lay.off_counts + 16 * 32 * 2 * 4
+    assert lay.bytes >= lay.off_lists + 16 * 32 * lay.list_cap * 4
+    assert dma.workspace_size(p) == lay.bytes
+    # window wider than the sequence: lists never exceed the padded sequence
+    lay2 = dma.workspace_layout(dma.make_params(B=1, H=1, Hkv=1, N=300, d=64, w=5000))
+    assert lay2.list_cap == 384 and lay2.n_blocks == 3
+    # decode: selection region
+    lay3 = dma.workspace_layout(dma.make_params(B=8, H=32, Hkv=8, N=65536, d=128, w=2048, Nq=1))
+    assert lay3.sel_len == 2048 and lay3.n_blocks == 0 and lay3.off_sel % 256 == 0
+
+
+# The fake-pointer checks run in a child process that sees no GPU, so a call
+# that wrongly passed validation could never launch a kernel on real memory.
+_FAKE_CHECKS = r"""
+import ctypes, sys
+sys.path.insert(0, %(root)r)
+import trainable_dynamic_mask_b200 as dma
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = 1 << 20   # 16-byte aligned, non-null, never dereferenced on the host
+lib = dma.load()
+def need_of(p):
+    n = ctypes.c_size_t(0)
+    assert lib.dma_workspace_size(ctypes.byref(p), ctypes.byref(n)) == OK
+    return n.value
+p = dma.make_params(1, 2, 1, 256, 64, 64)
+pp = ctypes.byref(p)
+need = need_of(p)
+assert lib.dma_gate(pp, None, FAKE, FAKE, FAKE, None, None, 0, None) == INVALID
+assert lib.dma_gate(pp, FAKE + 4, FAKE, FAKE, FAKE, None, None, 0, None) == INVALID
+assert lib.dma_gate(pp, FAKE, FAKE, FAKE, FAKE, FAKE + 8, None, 0, None) == INVALID
+assert lib.dma_topk_mask(pp, FAKE, FAKE, None, need, None) == WORKSPACE
+assert lib.dma_topk_mask(pp, FAKE, FAKE, FAKE, need - 1, None) == WORKSPACE
+assert lib.dma_topk_mask(pp, FAKE, FAKE, FAKE + 4, need, None) == WORKSPACE
+assert lib.dma_topk_mask(pp, FAKE, None, FAKE, need, None) == INVALID
+pd = dma.make_params(1, 2, 1, 256, 64, 64, Nq=1)
+needd = need_of(pd)
+assert lib.dma_topk_mask(ctypes.byref(pd), FAKE, FAKE, FAKE, needd, None) == INVALID
+assert lib.dma_attn_fwd(pp, FAKE, FAKE, FAKE, FAKE, None, FAKE, need, FAKE, FAKE, None) == INVALID
+# attn_bwd(p, Q, K, V, delta, evict, ws, ws_bytes, O, LSE, dO, dQ, dK, dV, d_delta, stream)
+args = [FAKE] * 6 + [needd] + [FAKE] * 7 + [None]
+assert len(args) == 15
+assert lib.dma_attn_bwd(ctypes.byref(pd), *args) == UNSUPPORTED
+args_bad = [FAKE] * 6 + [need] + [FAKE] * 6 + [None, None]
+assert len(args_bad) == 15
+assert lib.dma_attn_bwd(pp, *args_bad) == INVALID
+# gate_bwd(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, ws, ws_bytes, stream)
+assert lib.dma_gate_bwd(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
+print("ok")
+"""
+
+
+def test_null_and_misaligned_pointers_are_rejected_before_launch():
+    import subprocess
+    import sys
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", _FAKE_CHECKS % {"root": ROOT}], env=env,
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr
+
+
+def test_python_binding_raises_on_error_status():
+    p = dma.make_params(1, 2, 1, 256, 64, 0)
+    with pytest.raises(dma.DmaError, match="INVALID_ARG"):
+        dma.workspace_size(p)

@@ -1,0 +1,258 @@
+// C-ABI entry points of libdma: argument validation, workspace plan, dispatch to launchers.
+// Nothing is launched before every argument has been checked.
+#include <math.h>
+#include <string.h>
+
+#include "internal.h"
+
+using namespace dma;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+
+dma_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? DMA_OK : DMA_ERR_CUDA; }
+
+// Validates the workspace for plan P.
+dma_status_t check_ws(const Plan& P, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned16(ws)) return DMA_ERR_WORKSPACE;
+  if (ws_bytes < P.bytes) return DMA_ERR_WORKSPACE;
+  return DMA_OK;
+}
+
+}  // namespace
+
+namespace dma {
+
+dma_status_t make_plan(const dma_params_t* p, Plan* P) {
+  if (p == nullptr || P == nullptr) return DMA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->Hkv < 1 || p->N < 1 || p->Nq < 1 || p->d < 1 || p->w < 1)
+    return DMA_ERR_INVALID_ARG;
+  if (p->H % p->Hkv != 0) return DMA_ERR_INVALID_ARG;
+  if (p->dtype != DMA_BF16 && p->dtype != DMA_F32) return DMA_ERR_INVALID_ARG;
+  if (p->Nq != p->N && p->Nq != 1) return DMA_ERR_INVALID_ARG;
+  if (!(p->scale == p->scale) || isinf(p->scale)) return DMA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return DMA_ERR_UNSUPPORTED;
+  if ((int64_t)p->B * p->H > 65535) return DMA_ERR_UNSUPPORTED;
+  Plan& R = *P;
+  memset(&R, 0, sizeof(R));
+  R.B = p->B; R.H = p->H; R.Hkv = p->Hkv; R.N = p->N; R.Nq = p->Nq; R.d = p->d; R.w = p->w;
+  R.G = p->H / p->Hkv;
+  R.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
+  R.bf16 = p->dtype == DMA_BF16;
+  R.decode = (p->Nq == 1 && p->N > 1);
+  if (!R.decode && p->N > kTopwMaxN) return DMA_ERR_UNSUPPORTED;
+  if (R.decode && p->N > (1 << 24)) return DMA_ERR_UNSUPPORTED;
+
+  const size_t BH = (size_t)R.B * R.H;
+  const int minwn = R.w < R.N ? R.w : R.N;
+  R.n_blocks = (R.N + kBlockQ - 1) / kBlockQ;
+  {
+    size_t cap = align_up((size_t)minwn + kBlockQ, kBlockQ);
+    size_t ncap = align_up((size_t)R.N, kBlockQ);
+    R.list_cap = (int)(cap < ncap ? cap : ncap);
+  }
+  R.sel_len = minwn;
+  R.n_split = (R.sel_len + kDecodeSplit - 1) / kDecodeSplit;
+  R.n_slices = (R.N + kGateSlice - 1) / kGateSlice;
+
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  R.off_status = take(256);
+  if (!R.decode) {
+    R.off_counts = take(BH * R.n_blocks * 2 * sizeof(int32_t));
+    R.off_lists = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
+    R.off_rowD = take(BH * R.Nq * sizeof(float));
+  } else {
+    R.off_sel = take(BH * R.sel_len * sizeof(int32_t));
+    R.off_dec_part = take(BH * R.n_split * (size_t)(R.d + 2) * sizeof(float));
+  }
+  if (!R.bf16) {
+    R.off_q16 = take(BH * R.Nq * R.d * 2);
+    R.off_k16 = take((size_t)R.B * R.Hkv * R.N * R.d * 2);
+    R.off_v16 = take((size_t)R.B * R.Hkv * R.N * R.d * 2);
+    R.off_do16 = take(BH * R.Nq * R.d * 2);
+  }
+  R.off_gx = take(BH * R.N * sizeof(float));
+  R.off_dA_part = take(BH * ((R.N + 1023) / 1024) * sizeof(float));
+  R.off_dDelta_part = take((size_t)R.n_slices * R.B * R.Hkv * R.d * R.H * sizeof(float));
+  R.bytes = off;
+  return DMA_OK;
+}
+
+}  // namespace dma
+
+extern "C" {
+
+const char* dma_status_string(dma_status_t s) {
+  switch (s) {
+    case DMA_OK: return "DMA_OK";
+    case DMA_ERR_INVALID_ARG: return "DMA_ERR_INVALID_ARG: invalid argument";
+    case DMA_ERR_UNSUPPORTED: return "DMA_ERR_UNSUPPORTED: valid request outside implemented limits";
+    case DMA_ERR_WORKSPACE: return "DMA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case DMA_ERR_CUDA: return "DMA_ERR_CUDA: a CUDA launch failed";
+    case DMA_ERR_TIMEOUT: return "DMA_ERR_TIMEOUT: a device-side bounded wait gave up";
+  }
+  return "DMA_ERR_UNKNOWN";
+}
+
+int32_t dma_abi_version(void) { return DMA_ABI_VERSION; }
+
+dma_status_t dma_workspace_size(const dma_params_t* p, size_t* bytes) {
+  if (bytes == nullptr) return DMA_ERR_INVALID_ARG;
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  *bytes = P.bytes;
+  return DMA_OK;
+}
+
+dma_status_t dma_workspace_layout(const dma_params_t* p, dma_ws_layout_t* L) {
+  if (L == nullptr) return DMA_ERR_INVALID_ARG;
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  memset(L, 0, sizeof(*L));
+  L->bytes = P.bytes;
+  L->off_status = P.off_status;
+  L->off_counts = P.off_counts;
+  L->off_lists = P.off_lists;
+  L->off_sel = P.off_sel;
+  L->n_blocks = P.decode ? 0 : P.n_blocks;
+  L->list_cap = P.decode ? 0 : P.list_cap;
+  L->sel_len = P.decode ? P.sel_len : 0;
+  return DMA_OK;
+}
+
+dma_status_t dma_gate(const dma_params_t* p, const void* V, const void* Delta, const float* A,
+                      float* delta, float* x_save, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!ok_ptr(V) || !ok_ptr(Delta) || !ok_ptr(A) || !ok_ptr(delta)) return DMA_ERR_INVALID_ARG;
+  if (x_save != nullptr && !aligned16(x_save)) return DMA_ERR_INVALID_ARG;
+  return cuda_status(launch_gate_fwd(P, V, Delta, A, delta, x_save, (cudaStream_t)stream));
+}
+
+dma_status_t dma_topk_mask(const dma_params_t* p, const float* delta, int32_t* evict,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!ok_ptr(delta)) return DMA_ERR_INVALID_ARG;
+  if (P.decode ? (evict != nullptr) : !ok_ptr(evict)) return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (P.decode) return cuda_status(launch_topw_decode(P, delta, workspace, s));
+  return cuda_status(launch_topw_prefill(P, delta, evict, workspace, s));
+}
+
+dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
+                          const float* delta, const int32_t* evict, void* workspace,
+                          size_t workspace_bytes, void* O, float* LSE, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(delta) || !ok_ptr(O) || !ok_ptr(LSE))
+    return DMA_ERR_INVALID_ARG;
+  if (P.decode ? (evict != nullptr) : !ok_ptr(evict)) return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const uint16_t *q16 = (const uint16_t*)Q, *k16 = (const uint16_t*)K, *v16 = (const uint16_t*)V;
+  cudaError_t e = cudaSuccess;
+  if (!P.bf16) {
+    const size_t nq = (size_t)P.B * P.H * P.Nq * P.d, nk = (size_t)P.B * P.Hkv * P.N * P.d;
+    uint16_t* q = ws_ptr<uint16_t>(workspace, P.off_q16);
+    uint16_t* k = ws_ptr<uint16_t>(workspace, P.off_k16);
+    uint16_t* v = ws_ptr<uint16_t>(workspace, P.off_v16);
+    if ((e = launch_convert_f32_to_bf16((const float*)Q, q, nq, s)) != cudaSuccess) return DMA_ERR_CUDA;
+    if ((e = launch_convert_f32_to_bf16((const float*)K, k, nk, s)) != cudaSuccess) return DMA_ERR_CUDA;
+    if ((e = launch_convert_f32_to_bf16((const float*)V, v, nk, s)) != cudaSuccess) return DMA_ERR_CUDA;
+    q16 = q; k16 = k; v16 = v;
+  }
+  if (P.decode) e = launch_decode_attn(P, q16, k16, v16, delta, workspace, O, LSE, s);
+  else e = launch_attn_fwd(P, q16, k16, v16, delta, evict, workspace, O, LSE, s);
+  return cuda_status(e);
+}
+
+dma_status_t dma_attn_bwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
+                          const float* delta, const int32_t* evict, void* workspace,
+                          size_t workspace_bytes, const void* O, const float* LSE,
+                          const void* dO, void* dQ, void* dK, void* dV, float* d_delta,
+                          void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (P.decode) return DMA_ERR_UNSUPPORTED;
+  if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(delta) || !ok_ptr(evict) || !ok_ptr(O) ||
+      !ok_ptr(LSE) || !ok_ptr(dO) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !ok_ptr(d_delta))
+    return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const uint16_t *q16 = (const uint16_t*)Q, *k16 = (const uint16_t*)K, *v16 = (const uint16_t*)V,
+                 *do16 = (const uint16_t*)dO;
+  if (!P.bf16) {
+    const size_t nq = (size_t)P.B * P.H * P.Nq * P.d, nk = (size_t)P.B * P.Hkv * P.N * P.d;
+    uint16_t* q = ws_ptr<uint16_t>(workspace, P.off_q16);
+    uint16_t* k = ws_ptr<uint16_t>(workspace, P.off_k16);
+    uint16_t* v = ws_ptr<uint16_t>(workspace, P.off_v16);
+    uint16_t* g = ws_ptr<uint16_t>(workspace, P.off_do16);
+    if (launch_convert_f32_to_bf16((const float*)Q, q, nq, s) != cudaSuccess) return DMA_ERR_CUDA;
+    if (launch_convert_f32_to_bf16((const float*)K, k, nk, s) != cudaSuccess) return DMA_ERR_CUDA;
+    if (launch_convert_f32_to_bf16((const float*)V, v, nk, s) != cudaSuccess) return DMA_ERR_CUDA;
+    if (launch_convert_f32_to_bf16((const float*)dO, g, nq, s) != cudaSuccess) return DMA_ERR_CUDA;
+    q16 = q; k16 = k; v16 = v; do16 = g;
+  }
+  return cuda_status(launch_attn_bwd(P, q16, k16, v16, delta, evict, workspace, O, LSE, do16, dQ,
+                                     dK, dV, d_delta, s));
+}
+
+dma_status_t dma_gate_bwd(const dma_params_t* p, const void* V, const void* Delta,
+                          const float* A, const float* x_save, const float* delta,
+                          const float* d_delta, float* dDelta, float* dA, float* dV_gate,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!ok_ptr(V) || !ok_ptr(Delta) || !ok_ptr(A) || !ok_ptr(x_save) || !ok_ptr(delta) ||
+      !ok_ptr(d_delta) || !ok_ptr(dDelta) || !ok_ptr(dA) || !ok_ptr(dV_gate))
+    return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  return cuda_status(launch_gate_bwd(P, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate,
+                                     workspace, (cudaStream_t)stream));
+}
+
+dma_status_t dma_check_device_status(const dma_params_t* p, void* workspace, void* stream,
+                                     int32_t* code) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (workspace == nullptr || code == nullptr) return DMA_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws_ptr<int32_t>(workspace, P.off_status), sizeof(v),
+                      cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DMA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DMA_ERR_CUDA;
+  *code = v;
+  return v == 0 ? DMA_OK : DMA_ERR_TIMEOUT;
+}
+
+dma_status_t dma_clear_device_status(const dma_params_t* p, void* workspace, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (workspace == nullptr) return DMA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws_ptr<int32_t>(workspace, P.off_status), 0, sizeof(int32_t),
+                                     (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,283 @@
+// Gate kernels: delta = exp(A * softplus(v Delta)) and its backward.
+//
+// Source: "Trainable Dynamic Mask Sparse Attention" (HF blog), section "Dynamic Sparse Mask
+// Generation", delta equation ("Dynamic Weight Computation"); Delta and A are learnable, and the
+// method is trainable end to end (section "Gradient Flow Integrity").
+//
+// x[b,h,j] = sum_r v_j[r] Delta[r,h] with v_j the concatenation of the Hkv value heads at key
+// position j (r = g*d + c).  The contraction is narrow (H = 2..32 columns), so it runs on the FMA
+// pipe with float32 accumulation: bf16 products are exact in float32, and float32 inputs keep
+// their full precision.  Each CTA stages a 64-position tile of one value head, transposed to
+// [channel][position], plus the matching Delta rows, and each thread accumulates a 4x4
+// (position x head) register tile.
+#include "common.cuh"
+
+namespace dma {
+namespace {
+
+constexpr int kGatePT = 64;  // positions per CTA
+
+DMA_DEVINL float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
+DMA_DEVINL float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
+
+template <typename T>
+__global__ void gate_fwd_kernel(const T* __restrict__ V, const T* __restrict__ Delta,
+                                const float* __restrict__ A, float* __restrict__ delta,
+                                float* __restrict__ x_save, int H, int Hkv, int N, int d,
+                                int H_pad) {
+  extern __shared__ float sm[];
+  float* Vs = sm;                    // [d][kGatePT]
+  float* Ds = sm + d * kGatePT;      // [d][H_pad]
+  const int b = blockIdx.y;
+  const int p0 = blockIdx.x * kGatePT;
+  const int TH = H_pad / 4;
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int tp = tid / TH, th = tid % TH;   // 16 position groups x TH head groups
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int g = 0; g < Hkv; ++g) {
+    const T* Vg = V + ((size_t)(b * Hkv + g) * N) * d;
+    for (int e = tid; e < kGatePT * d; e += nth) {
+      int p = e / d, c = e % d;
+      int pos = p0 + p;
+      Vs[c * kGatePT + p] = pos < N ? load_as_f32(Vg + (size_t)pos * d + c) : 0.f;
+    }
+    for (int e = tid; e < d * H_pad; e += nth) {
+      int c = e / H_pad, h = e % H_pad;
+      Ds[e] = h < H ? load_as_f32(Delta + (size_t)(g * d + c) * H + h) : 0.f;
+    }
+    __syncthreads();
+    for (int c = 0; c < d; ++c) {
+      float4 v4 = *reinterpret_cast<const float4*>(Vs + c * kGatePT + tp * 4);
+      float4 d4 = *reinterpret_cast<const float4*>(Ds + c * H_pad + th * 4);
+      float vv[4] = {v4.x, v4.y, v4.z, v4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(vv[i], dd[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int h = th * 4 + j;
+    if (h >= H) continue;
+    const float a = A[h];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int pos = p0 + tp * 4 + i;
+      if (pos >= N) continue;
+      const float x = acc[i][j];
+      const size_t o = (size_t)(b * H + h) * N + pos;
+      delta[o] = expf(a * softplus_f(x));
+      if (x_save) x_save[o] = x;
+    }
+  }
+}
+
+__global__ void convert_f32_bf16_kernel(const float* __restrict__ src, uint16_t* __restrict__ dst,
+                                        size_t n) {
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  const size_t n4 = n / 4;
+  for (size_t k = i; k < n4; k += stride) {
+    float4 v = reinterpret_cast<const float4*>(src)[k];
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    reinterpret_cast<uint2*>(dst)[k] = o;
+  }
+  for (size_t k = n4 * 4 + i; k < n; k += stride) dst[k] = f32_to_bf16(src[k]);
+}
+
+// ---------------------------------------------------------------- backward
+
+// gx = d_delta * delta * A * sigmoid(x); partial sums of d_delta * delta * softplus(x) for dA.
+__global__ void gate_bwd_pointwise_kernel(const float* __restrict__ x, const float* __restrict__ delta,
+                                          const float* __restrict__ dd, const float* __restrict__ A,
+                                          float* __restrict__ gx, float* __restrict__ dA_part,
+                                          int H, int N) {
+  __shared__ float red[32];
+  const int row = blockIdx.y;   // b*H + h
+  const int h = row % H;
+  const float a = A[h];
+  const size_t base = (size_t)row * N;
+  float part = 0.f;
+  for (int k = 0; k < 4; ++k) {
+    const int j = blockIdx.x * 1024 + k * 256 + threadIdx.x;
+    if (j < N) {
+      const float xv = x[base + j], dv = delta[base + j], g = dd[base + j];
+      gx[base + j] = g * dv * a * sigmoid_f(xv);
+      part += g * dv * softplus_f(xv);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = part;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) dA_part[(size_t)row * gridDim.x + blockIdx.x] = v;
+  }
+}
+
+// dV_gate[b,g,j,c] = sum_h gx[b,h,j] * Delta[g*d+c, h]
+template <typename T>
+__global__ void gate_bwd_dv_kernel(const float* __restrict__ gx, const T* __restrict__ Delta,
+                                   float* __restrict__ dVg, int H, int Hkv, int N, int d) {
+  extern __shared__ float sm[];
+  float* Gs = sm;                 // [H][kGatePT]
+  float* Ds = sm + H * kGatePT;   // [d][H]
+  const int b = blockIdx.y, j0 = blockIdx.x * kGatePT;
+  for (int e = threadIdx.x; e < H * kGatePT; e += blockDim.x) {
+    int h = e / kGatePT, p = e % kGatePT;
+    Gs[e] = (j0 + p < N) ? gx[(size_t)(b * H + h) * N + j0 + p] : 0.f;
+  }
+  for (int g = 0; g < Hkv; ++g) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < d * H; e += blockDim.x) Ds[e] = load_as_f32(Delta + (size_t)g * d * H + e);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kGatePT * d; e += blockDim.x) {
+      const int p = e / d, c = e % d;
+      if (j0 + p >= N) continue;
+      float acc = 0.f;
+      for (int h = 0; h < H; ++h) acc = fmaf(Gs[h * kGatePT + p], Ds[c * H + h], acc);
+      dVg[((size_t)(b * Hkv + g) * N + j0 + p) * d + c] = acc;
+    }
+  }
+}
+
+// partial[(s*B + b)][g*d + c][h] = sum_{j in slice s} V[b,g,j,c] * gx[b,h,j]
+template <typename T>
+__global__ void gate_bwd_ddelta_partial_kernel(const T* __restrict__ V, const float* __restrict__ gx,
+                                               float* __restrict__ part, int B, int H, int Hkv,
+                                               int N, int d) {
+  extern __shared__ float sm[];
+  float* Vs = sm;                   // [64][d]
+  float* Gs = sm + 64 * d;          // [H][64]
+  const int s = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
+  const int c = threadIdx.x % d;
+  const int hg = threadIdx.x / d, nhg = blockDim.x / d;
+  float acc[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+  const T* Vg = V + (size_t)(b * Hkv + g) * N * d;
+  for (int j0 = s * kGateSlice; j0 < min(N, (s + 1) * kGateSlice); j0 += 64) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 64 * d; e += blockDim.x) {
+      const int p = e / d, cc = e % d;
+      Vs[e] = (j0 + p < N) ? load_as_f32(Vg + (size_t)(j0 + p) * d + cc) : 0.f;
+    }
+    for (int e = threadIdx.x; e < H * 64; e += blockDim.x) {
+      const int h = e / 64, p = e % 64;
+      Gs[e] = (j0 + p < N) ? gx[(size_t)(b * H + h) * N + j0 + p] : 0.f;
+    }
+    __syncthreads();
+    for (int p = 0; p < 64; ++p) {
+      const float v = Vs[p * d + c];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        const int h = hg + k * nhg;
+        if (h < H) acc[k] = fmaf(v, Gs[h * 64 + p], acc[k]);
+      }
+    }
+  }
+  float* out = part + ((size_t)(s * B + b) * Hkv * d + (size_t)g * d + c) * H;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int h = hg + k * nhg;
+    if (h < H) out[h] = acc[k];
+  }
+}
+
+__global__ void gate_bwd_reduce_kernel(const float* __restrict__ part, const float* __restrict__ dA_part,
+                                       float* __restrict__ dDelta, float* __restrict__ dA, int nparts,
+                                       int RH, int H, int B, int nchunk) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < RH) {
+    float acc = 0.f;
+    for (int k = 0; k < nparts; ++k) acc += part[(size_t)k * RH + i];
+    dDelta[i] = acc;
+  }
+  if (i < H) {
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b)
+      for (int k = 0; k < nchunk; ++k) acc += dA_part[((size_t)b * H + i) * nchunk + k];
+    dA[i] = acc;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
+                            float* delta, float* x_save, cudaStream_t s) {
+  const int H_pad = (P.H + 3) / 4 * 4;
+  const int threads = 16 * (H_pad / 4);
+  if (threads > 1024) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)(P.d * kGatePT + P.d * H_pad) * sizeof(float);
+  dim3 grid((P.N + kGatePT - 1) / kGatePT, P.B);
+  if (P.bf16) {
+    auto k = gate_fwd_kernel<uint16_t>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, threads, smem, s>>>((const uint16_t*)V, (const uint16_t*)Delta, A, delta, x_save, P.H,
+                                  P.Hkv, P.N, P.d, H_pad);
+  } else {
+    auto k = gate_fwd_kernel<float>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, threads, smem, s>>>((const float*)V, (const float*)Delta, A, delta, x_save, P.H, P.Hkv,
+                                  P.N, P.d, H_pad);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  size_t blocks = (n / 4 + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  if (blocks == 0) blocks = 1;
+  convert_f32_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, const float* A,
+                            const float* x_save, const float* delta, const float* d_delta,
+                            float* dDelta, float* dA, float* dV_gate, void* ws, cudaStream_t s) {
+  if (P.H > 32 * (256 / P.d)) return cudaErrorInvalidValue;
+  float* gx = ws_ptr<float>(ws, P.off_gx);
+  float* dA_part = ws_ptr<float>(ws, P.off_dA_part);
+  float* part = ws_ptr<float>(ws, P.off_dDelta_part);
+  const int nchunk = (P.N + 1023) / 1024;
+  gate_bwd_pointwise_kernel<<<dim3(nchunk, P.B * P.H), 256, 0, s>>>(x_save, delta, d_delta, A, gx,
+                                                                     dA_part, P.H, P.N);
+  const size_t smem_dv = (size_t)(P.H * kGatePT + P.d * P.H) * sizeof(float);
+  const size_t smem_dd = (size_t)(64 * P.d + P.H * 64) * sizeof(float);
+  dim3 gdv((P.N + kGatePT - 1) / kGatePT, P.B);
+  dim3 gdd(P.n_slices, P.B, P.Hkv);
+  if (P.bf16) {
+    auto k1 = gate_bwd_dv_kernel<uint16_t>;
+    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dv);
+    k1<<<gdv, 256, smem_dv, s>>>(gx, (const uint16_t*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
+    auto k2 = gate_bwd_ddelta_partial_kernel<uint16_t>;
+    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dd);
+    k2<<<gdd, 256, smem_dd, s>>>((const uint16_t*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
+  } else {
+    auto k1 = gate_bwd_dv_kernel<float>;
+    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dv);
+    k1<<<gdv, 256, smem_dv, s>>>(gx, (const float*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
+    auto k2 = gate_bwd_ddelta_partial_kernel<float>;
+    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dd);
+    k2<<<gdd, 256, smem_dd, s>>>((const float*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
+  }
+  const int RH = P.Hkv * P.d * P.H;
+  gate_bwd_reduce_kernel<<<(RH + 255) / 256, 256, 0, s>>>(part, dA_part, dDelta, dA,
+                                                          P.n_slices * P.B, RH, P.H, P.B, nchunk);
+  return cudaGetLastError();
+}
+
+}  // namespace dma

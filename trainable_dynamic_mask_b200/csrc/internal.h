@@ -1,0 +1,68 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernel launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dma.h"
+
+namespace dma {
+
+constexpr int kBlockQ = DMA_BLOCK_Q;   // query rows per block of the mask encoding
+constexpr int kTopwMaxN = 16384;      // prefill/training selection keeps a whole row in SMEM
+constexpr int kDecodeSplit = 256;      // selected keys per decode split
+constexpr int kGateSlice = 512;        // positions per partial sum of dDelta
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Resolved problem and workspace plan.
+struct Plan {
+  int B, H, Hkv, N, Nq, d, w, G;
+  float scale;
+  bool bf16;      // storage dtype is bf16 (else f32)
+  bool decode;    // Nq == 1 and N > 1 ... the single query sits at position N-1
+  int n_blocks;   // query blocks of kBlockQ rows (prefill)
+  int list_cap;   // entries per block list
+  int sel_len;    // decode: min(w, N)
+  int n_split;    // decode: splits per (b, h)
+  int n_slices;   // gate backward: position slices of kGateSlice
+  // byte offsets in the workspace
+  size_t off_status, off_counts, off_lists, off_sel;
+  size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
+  size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
+  size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
+  size_t off_gx;                       // gate backward: gx [B, H, N] f32
+  size_t off_dA_part;                  // gate backward: [B*H][ceil(N/1024)] f32
+  size_t off_dDelta_part;              // gate backward: [n_slices*B][Hkv*d][H] f32
+  size_t bytes;
+};
+
+dma_status_t make_plan(const dma_params_t* p, Plan* plan);
+
+template <typename T> inline T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- launchers (cudaError_t)
+cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
+                            float* delta, float* x_save, cudaStream_t s);
+cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evict, void* ws,
+                                cudaStream_t s);
+cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s);
+cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t s);
+cudaError_t launch_attn_fwd(const Plan& P, const uint16_t* Q, const uint16_t* K,
+                            const uint16_t* V, const float* delta, const int32_t* evict,
+                            void* ws, void* O, float* LSE, cudaStream_t s);
+cudaError_t launch_decode_attn(const Plan& P, const uint16_t* Q, const uint16_t* K,
+                               const uint16_t* V, const float* delta, void* ws, void* O,
+                               float* LSE, cudaStream_t s);
+cudaError_t launch_attn_bwd(const Plan& P, const uint16_t* Q, const uint16_t* K,
+                            const uint16_t* V, const float* delta, const int32_t* evict,
+                            void* ws, const void* O, const float* LSE, const uint16_t* dO16,
+                            void* dQ, void* dK, void* dV, float* d_delta, cudaStream_t s);
+cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, const float* A,
+                            const float* x_save, const float* delta, const float* d_delta,
+                            float* dDelta, float* dA, float* dV_gate, void* ws, cudaStream_t s);
+
+}  // namespace dma
