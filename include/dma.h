@@ -99,12 +99,15 @@ typedef struct {
  * dma_workspace_size() bytes, passed to every call of one problem.  Its leading regions are
  * part of the ABI so that callers and tests can read the mask encoding:
  *
- *   off_status  int32 device status word (0 = ok), written by bounded waits.
+ *   off_status  int32 device status word (0 = ok): kernels OR an error code into it (a bounded
+ *               wait that gave up, an internal consistency check that failed).  Its content in a
+ *               new workspace is undefined: clear it once with dma_clear_device_status.
  *   off_counts  int32 [B, H, n_blocks, 2]: per query block, (n_full, n_live).
- *   off_lists   int32 [B, H, n_blocks, list_cap]: the live keys of each query block, the
- *               n_full "full" keys (selected by every row of the block) first, then the
- *               partial ones; each group in ascending key order.  Entries past n_live are
- *               unspecified.
+ *   off_lists   int32 [B, H, n_blocks, list_cap]: the live keys of each query block
+ *               [t0, t1), t1 = min(t0 + DMA_BLOCK_Q, N): first the n_full "full" keys, selected
+ *               by every row of the block (j <= t0 and e_j >= t1), then the partial ones (at
+ *               most 2*DMA_BLOCK_Q); each group in ascending key order.  Entries past n_live
+ *               are unspecified.
  *   off_sel     decode only: int32 [B, H, sel_len] selected keys of the query, ascending.
  *   the rest    internal scratch.
  */

@@ -184,9 +184,8 @@ def live_keys_per_block(e: np.ndarray, Bq: int):
     (selected by every query row of the block) and 'partial' keys.
 
     Returns a list over blocks of (full: sorted int array, partial: sorted int
-    array).  A key is full when j <= t0 and e_j >= t0 + Bq (so in a ragged
-    last block, where rows past N do not exist, surviving keys still count as
-    partial: they are masked, which is always correct).
+    array).  A key is full when every existing row of the block selects it:
+    j <= t0 and e_j >= t1 with t1 = min(t0 + Bq, N) (rows past N do not exist).
     """
     N = e.shape[0]
     j = np.arange(N)
@@ -194,7 +193,7 @@ def live_keys_per_block(e: np.ndarray, Bq: int):
     for t0 in range(0, N, Bq):
         t1 = min(t0 + Bq, N)
         live = (j < t1) & (e > np.maximum(j, t0))
-        full = live & (j <= t0) & (e >= t0 + Bq)
+        full = live & (j <= t0) & (e >= t1)
         out.append((np.nonzero(full)[0], np.nonzero(live & ~full)[0]))
     return out
 

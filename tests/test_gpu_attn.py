@@ -15,12 +15,12 @@ from gpu_common import assert_close, f32_dev, lib, to_dev, to_np, torch_cuda
 pytestmark = pytest.mark.gpu
 
 
-def _setup(wl, with_dO=False):
+def _setup(wl, with_dO=False, bf16_values=False):
     """Inputs on both sides, the oracle's delta and eviction index, and the
     GPU mask built from that delta."""
     dma = lib()
     torch = torch_cuda()
-    I = make_inputs(wl, with_dO=with_dO)
+    I = make_inputs(wl, with_dO=with_dO, bf16_values=bf16_values)
     big = wl.N * wl.B > 4096
     _, d64 = oracle.gate(I.V, I.Delta, I.A, gemm_dtype=np.float32 if big else np.float64)
     d32 = d64.astype(np.float32)
@@ -117,8 +117,12 @@ def _bwd(dma, torch, wl, p, ws, dev, O, LSE):
 
 @pytest.mark.parametrize("case", list(BWD_CASES))
 def test_attn_bwd_full(case):
+    """For float32 storage the attention kernels round Q, K, V and dO to bf16
+    when they load them; the backward check feeds bf16-representable float32
+    values so that it measures the kernels' arithmetic against the tolerance
+    (the float32 forward is checked on unrounded values above)."""
     wl = BWD_CASES[case]
-    dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl, with_dO=True)
+    dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl, with_dO=True, bf16_values=True)
     O, LSE = _fwd(dma, torch, wl, p, ws, dev)
     dQ, dK, dV, dd = _bwd(dma, torch, wl, p, ws, dev, O, LSE)
     r = oracle.attn_bwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, I.dO)
@@ -207,7 +211,7 @@ def test_forward_backward_chain_on_tiny():
     dma = lib()
     torch = torch_cuda()
     wl = get("tiny")
-    I = make_inputs(wl, with_dO=True)
+    I = make_inputs(wl, with_dO=True, bf16_values=True)   # see test_attn_bwd_full
     p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype=wl.dtype)
     Q, K, V = f32_dev(I.Q), f32_dev(I.K), f32_dev(I.V)
     Dl, A, dO = f32_dev(I.Delta), f32_dev(I.A), f32_dev(I.dO)

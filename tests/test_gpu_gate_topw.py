@@ -55,6 +55,7 @@ def _topw_case(B, H, N, w, delta_np):
     torch = torch_cuda()
     p = dma.make_params(B, H, H, N, 64, w)
     ws = torch.empty(dma.workspace_size(p), dtype=torch.uint8, device="cuda")
+    dma.clear_device_status(p, ws)
     delta = f32_dev(delta_np)
     evict = torch.full((B, H, N), -7, dtype=torch.int32, device="cuda")
     dma.topk_mask(p, delta, evict, ws)

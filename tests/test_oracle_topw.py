@@ -85,9 +85,10 @@ def test_window_at_least_N_keeps_all_causal_keys():
         np.testing.assert_array_equal(oracle.topw_eviction(delta, w), np.full(N, N))
 
 
-def test_live_keys_per_block_against_mask():
-    N, w, Bq = 203, 31, 16
-    for kind in ("uniform", "levels", "increasing"):
+@pytest.mark.parametrize("N,w", [(203, 31), (203, 500), (100, 16), (64, 64)])
+def test_live_keys_per_block_against_mask(N, w):
+    Bq = 16
+    for kind in ("uniform", "levels", "increasing", "constant"):
         delta = make_delta((N,), seed=2, kind=kind, levels=4)
         M = oracle.topw_sets_bruteforce(delta, w)
         e = oracle.topw_eviction(delta, w)
@@ -98,8 +99,8 @@ def test_live_keys_per_block_against_mask():
             union = M[t0:t1].any(axis=0)
             inter = M[t0:t1].all(axis=0)
             np.testing.assert_array_equal(np.sort(np.concatenate([full, partial])), np.nonzero(union)[0])
-            if t1 - t0 == Bq:
-                np.testing.assert_array_equal(full, np.nonzero(inter)[0])
+            np.testing.assert_array_equal(full, np.nonzero(inter)[0])
             assert set(full).isdisjoint(partial)
-            # the live set never exceeds w + Bq keys
+            # the live set never exceeds w + Bq keys, the partial keys never 2 Bq
             assert full.size + partial.size <= w + Bq
+            assert partial.size <= 2 * Bq

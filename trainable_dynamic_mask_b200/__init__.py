@@ -19,7 +19,8 @@ from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DmaError, DmaParams, DmaWsLayout,
 __all__ = [
     "BLOCK_Q", "DMA_BF16", "DMA_F32", "DmaError", "DmaParams", "LIB_PATH", "load", "exported_names",
     "make_params", "workspace_size", "workspace_layout", "gate", "topk_mask", "attn_fwd", "attn_bwd",
-    "gate_bwd", "check_device_status", "clear_device_status", "abi_version", "forward", "backward",
+    "gate_bwd", "check_device_status", "clear_device_status", "abi_version", "alloc_workspace", "forward",
+    "backward",
 ]
 
 
@@ -114,9 +115,12 @@ def clear_device_status(p, workspace, stream=None):
 
 # ---------------------------------------------------------------- convenience (torch allocation)
 
-def _alloc(p, device):
+def alloc_workspace(p, device="cuda", stream=None):
+    """A workspace for problem p (torch allocation) with its status word cleared."""
     import torch
-    return torch.empty(workspace_size(p), dtype=torch.uint8, device=device)
+    ws = torch.empty(workspace_size(p), dtype=torch.uint8, device=device)
+    clear_device_status(p, ws, stream)
+    return ws
 
 
 def forward(p, Q, K, V, Delta, A, workspace=None, stream=None):
@@ -125,7 +129,7 @@ def forward(p, Q, K, V, Delta, A, workspace=None, stream=None):
     delta, x, evict (None for decode), O, LSE, workspace."""
     import torch
     dev = Q.device
-    ws = workspace if workspace is not None else _alloc(p, dev)
+    ws = workspace if workspace is not None else alloc_workspace(p, dev, stream)
     f32 = torch.float32
     delta = torch.empty((p.B, p.H, p.N), dtype=f32, device=dev)
     x = torch.empty((p.B, p.H, p.N), dtype=f32, device=dev)

@@ -3,6 +3,11 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "common.cuh"
 #include "internal.h"
 
 using namespace dma;
@@ -24,6 +29,19 @@ dma_status_t check_ws(const Plan& P, const void* ws, size_t ws_bytes) {
 }  // namespace
 
 namespace dma {
+
+cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert({kernel, dev});
+  return e;
+}
 
 dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   if (p == nullptr || P == nullptr) return DMA_ERR_INVALID_ARG;

@@ -461,7 +461,7 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
   {
     auto k = bwd_dq_kernel<D, OutT>;
     const int smem = DqSmem<D>::kBytes;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
     k<<<dim3(P.n_blocks, P.B * P.H), kDqThreads, smem, s>>>(
         Q, K, V, dO, delta, evict, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists), LSE,
         Drow, (OutT*)dQ, P.H, P.G, P.N, P.n_blocks, P.list_cap, P.scale * kLog2e, P.scale);
@@ -469,7 +469,7 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
   {
     auto k = bwd_dkv_kernel<D, OutT>;
     const int smem = DkvSmem<D>::kBytes;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
     k<<<dim3((P.N + 63) / 64, P.B * P.Hkv), kDkvThreads, smem, s>>>(
         Q, K, V, dO, delta, evict, LSE, Drow, (OutT*)dK, (OutT*)dV, d_delta, P.H, P.G, P.N,
         P.scale * kLog2e, P.scale);

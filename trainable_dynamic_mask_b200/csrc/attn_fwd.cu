@@ -392,7 +392,7 @@ cudaError_t launch_fwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
                          cudaStream_t s) {
   auto k = attn_fwd_kernel<D, OutT>;
   const int smem = FwdSmem<D>::kBytes;
-  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
   dim3 grid(P.n_blocks, P.B * P.H);
   k<<<grid, kFwdThreads, smem, s>>>(Q, K, V, delta, evict, ws_ptr<int32_t>(ws, P.off_counts),
                                     ws_ptr<int32_t>(ws, P.off_lists), (OutT*)O, LSE, P.H, P.G, P.N,

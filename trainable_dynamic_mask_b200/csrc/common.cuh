@@ -92,6 +92,15 @@ DMA_DEVINL uint32_t swz(int r, int c, int row_chunks) {
   return (uint32_t)((r * row_chunks + (c ^ (r & 7))) * 16);
 }
 
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device) -- the attribute lives
+// in the device context -- so that no such call happens while a caller captures a stream into a
+// CUDA graph.
+cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes);
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel k, int bytes) {
+  return ensure_smem_limit_impl(reinterpret_cast<const void*>(k), bytes);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -224,12 +224,12 @@ cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, con
   dim3 grid((P.N + kGatePT - 1) / kGatePT, P.B);
   if (P.bf16) {
     auto k = gate_fwd_kernel<uint16_t>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    { cudaError_t ea = ensure_smem_limit(k, (int)smem); if (ea != cudaSuccess) return ea; }
     k<<<grid, threads, smem, s>>>((const uint16_t*)V, (const uint16_t*)Delta, A, delta, x_save, P.H,
                                   P.Hkv, P.N, P.d, H_pad);
   } else {
     auto k = gate_fwd_kernel<float>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    { cudaError_t ea = ensure_smem_limit(k, (int)smem); if (ea != cudaSuccess) return ea; }
     k<<<grid, threads, smem, s>>>((const float*)V, (const float*)Delta, A, delta, x_save, P.H, P.Hkv,
                                   P.N, P.d, H_pad);
   }
@@ -261,17 +261,17 @@ cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, con
   dim3 gdd(P.n_slices, P.B, P.Hkv);
   if (P.bf16) {
     auto k1 = gate_bwd_dv_kernel<uint16_t>;
-    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dv);
+    { cudaError_t ea = ensure_smem_limit(k1, (int)smem_dv); if (ea != cudaSuccess) return ea; }
     k1<<<gdv, 256, smem_dv, s>>>(gx, (const uint16_t*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
     auto k2 = gate_bwd_ddelta_partial_kernel<uint16_t>;
-    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dd);
+    { cudaError_t ea = ensure_smem_limit(k2, (int)smem_dd); if (ea != cudaSuccess) return ea; }
     k2<<<gdd, 256, smem_dd, s>>>((const uint16_t*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
   } else {
     auto k1 = gate_bwd_dv_kernel<float>;
-    cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dv);
+    { cudaError_t ea = ensure_smem_limit(k1, (int)smem_dv); if (ea != cudaSuccess) return ea; }
     k1<<<gdv, 256, smem_dv, s>>>(gx, (const float*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
     auto k2 = gate_bwd_ddelta_partial_kernel<float>;
-    cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dd);
+    { cudaError_t ea = ensure_smem_limit(k2, (int)smem_dd); if (ea != cudaSuccess) return ea; }
     k2<<<gdd, 256, smem_dd, s>>>((const float*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
   }
   const int RH = P.Hkv * P.d * P.H;

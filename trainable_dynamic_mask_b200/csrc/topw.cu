@@ -21,7 +21,9 @@
 //     keys better than r follows from T_k and the sorted candidate list.  New keys that survive to
 //     the end (rank <= T at the last boundary) get e = N.  Every key's e is written exactly once.
 // A second kernel (one CTA per (row, query block)) compacts the live keys of each block:
-// full keys (j <= t0 and e_j >= t0 + C) first, then the partial ones, each in ascending order.
+// full keys (selected by every existing row: j <= t0 and e_j >= min(t0 + C, N)) first, then the
+// partial ones (at most 2C: keys evicted inside the block and the block's own keys), each in
+// ascending order.
 #include "common.cuh"
 
 namespace dma {
@@ -281,7 +283,7 @@ topw_rows_kernel(const float* __restrict__ delta, int32_t* __restrict__ evict,
   }
 }
 
-// Live keys of query block k: j < t1 and e_j > max(j, t0).  Full keys first.
+// Live keys of query block k: j < t1 and e_j > max(j, t0).  Full keys (j <= t0, e_j >= t1) first.
 constexpr int kListThreads = 256;
 
 __global__ void __launch_bounds__(kListThreads)
@@ -303,7 +305,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ count
       const int j = base + tid * 4 + u;
       int e = j < t1 ? erow[j] : 0;
       const bool live = j < t1 && e > max(j, t0);
-      const bool full = live && j <= t0 && e >= t0 + kC;
+      const bool full = live && j <= t0 && e >= t1;
       f[u] = full;
       q[u] = live && !full;
       cf += f[u];
@@ -463,7 +465,7 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   const int rows = P.B * P.H;
   size_t smem = topw_rows_smem_bytes(P.N);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaFuncSetAttribute(topw_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  { cudaError_t ea = ensure_smem_limit(topw_rows_kernel, (int)smem); if (ea != cudaSuccess) return ea; }
   topw_rows_kernel<<<rows, kSortThreads, smem, s>>>(delta, evict, ws_ptr<int32_t>(ws, P.off_status),
                                                    P.N, P.w);
   topw_lists_kernel<<<dim3(P.n_blocks, rows), kListThreads, 0, s>>>(

@@ -72,6 +72,10 @@ class Workload:
         return int(np.minimum(t + 1, self.w).sum()) * self.B * self.H
 
     def with_(self, **kw) -> "Workload":
+        """A copy with some fields changed.  Changing N keeps the query-row
+        mode: prefill/train (Nq == N) follows the new N, decode keeps Nq = 1."""
+        if "N" in kw and "Nq" not in kw:
+            kw["Nq"] = 1 if self.Nq == 1 and self.N > 1 else kw["N"]
         return replace(self, **kw)
 
 
@@ -141,9 +145,12 @@ def _normal(rng: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
     return x
 
 
-def make_inputs(wl: Workload, with_dO: bool | None = None) -> Inputs:
+def make_inputs(wl: Workload, with_dO: bool | None = None, bf16_values: bool = False) -> Inputs:
     """Draw the inputs of `wl` from numpy's default_rng(seed) in the fixed
-    order Q, K, V, Delta, A, scaled positions, dO."""
+    order Q, K, V, Delta, A, scaled positions, dO.
+
+    bf16_values: for dtype "f32", round Q, K, V, Delta and dO to
+    bf16-representable values (still stored as float32)."""
     if with_dO is None:
         with_dO = wl.with_dO
     rng = np.random.default_rng(wl.seed)
@@ -169,7 +176,12 @@ def make_inputs(wl: Workload, with_dO: bool | None = None) -> Inputs:
         Delta, bits["Delta"] = bf16_round(Delta)
         if dO is not None:
             dO, bits["dO"] = bf16_round(dO)
-    elif wl.dtype != "f32":
+    elif wl.dtype == "f32":
+        if bf16_values:
+            Q, K, V, Delta = (bf16_round(a)[0] for a in (Q, K, V, Delta))
+            if dO is not None:
+                dO = bf16_round(dO)[0]
+    else:
         raise ValueError(f"unknown dtype {wl.dtype}")
     return Inputs(Q=Q, K=K, V=V, Delta=Delta, A=A, scaled_pos=pos, dO=dO, bits=bits)
 
