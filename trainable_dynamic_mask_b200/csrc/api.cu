@@ -31,6 +31,8 @@ dma_status_t check_ws(const Plan& P, const void* ws, size_t ws_bytes) {
 namespace dma {
 
 cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
+  // The limit is raised to the device's opt-in maximum (minus the kernel's static shared memory)
+  // the first time a kernel is launched on a device, whatever this launch needs.
   static std::mutex mu;
   static std::set<std::pair<const void*, int>> done;
   int dev = 0;
@@ -38,7 +40,13 @@ cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
   if (done.count({kernel, dev})) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  int optin = 0;
+  if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+  const int limit = optin - (int)fa.sharedSizeBytes;
+  if (bytes > limit) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, limit);
   if (e == cudaSuccess) done.insert({kernel, dev});
   return e;
 }

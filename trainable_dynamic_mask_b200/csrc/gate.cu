@@ -15,67 +15,111 @@
 namespace dma {
 namespace {
 
-constexpr int kGatePT = 64;  // positions per CTA
+constexpr int kGatePT = 64;  // positions per CTA (backward kernels)
+
+// 8 consecutive elements (16-byte aligned) widened to float.
+DMA_DEVINL void load8_as_f32(const uint16_t* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+DMA_DEVINL void load8_as_f32(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 
 DMA_DEVINL float softplus_f(float x) { return fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))); }
 DMA_DEVINL float sigmoid_f(float x) { return 1.f / (1.f + expf(-x)); }
 
-template <typename T>
-__global__ void gate_fwd_kernel(const T* __restrict__ V, const T* __restrict__ Delta,
-                                const float* __restrict__ A, float* __restrict__ delta,
-                                float* __restrict__ x_save, int H, int Hkv, int N, int d,
-                                int H_pad) {
-  extern __shared__ float sm[];
-  float* Vs = sm;                    // [d][kGatePT]
-  float* Ds = sm + d * kGatePT;      // [d][H_pad]
-  const int b = blockIdx.y;
-  const int p0 = blockIdx.x * kGatePT;
-  const int TH = H_pad / 4;
-  const int tid = threadIdx.x, nth = blockDim.x;
-  const int tp = tid / TH, th = tid % TH;   // 16 position groups x TH head groups
-  float acc[4][4];
+// CTA = 32 key positions of one batch row, 256 threads = 8 reduction groups x 32 threads.  The
+// reduction dimension r = g*d + c is processed in chunks of kGateR; inside a chunk group k takes
+// r = k, k+8, ...  Each thread holds a 4-position x HPT-head register tile (thread = 8 position
+// groups x 4 head groups); the 8 partial tiles are summed through shared memory at the end.
+constexpr int kGateP = 32;      // positions per CTA
+constexpr int kGateR = 256;     // reduction rows staged per chunk
+constexpr int kGateThreads = 256;
+
+template <typename T, int HPT>
+__global__ void __launch_bounds__(kGateThreads)
+gate_fwd_kernel(const T* __restrict__ V, const T* __restrict__ Delta, const float* __restrict__ A,
+                float* __restrict__ delta, float* __restrict__ x_save, int H, int Hkv, int N, int d) {
+  constexpr int HP = 4 * HPT;                       // padded head count
+  extern __shared__ __align__(16) float sm[];
+  float* Vt = sm;                                   // [kGateR][kGateP]   V transposed
+  float* Ds = Vt + kGateR * kGateP;                 // [kGateR][HP]
+  float* red = Ds + kGateR * HP;                    // [8][kGateP][HP]
+  const int b = blockIdx.y, p0 = blockIdx.x * kGateP;
+  const int tid = threadIdx.x, kg = tid >> 5, lane = tid & 31;
+  const int pg = lane & 7, hg = lane >> 3;
+  const int R = Hkv * d;
+  float acc[4][HPT];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < HPT; ++j) acc[i][j] = 0.f;
 
-  for (int g = 0; g < Hkv; ++g) {
-    const T* Vg = V + ((size_t)(b * Hkv + g) * N) * d;
-    for (int e = tid; e < kGatePT * d; e += nth) {
-      int p = e / d, c = e % d;
-      int pos = p0 + p;
-      Vs[c * kGatePT + p] = pos < N ? load_as_f32(Vg + (size_t)pos * d + c) : 0.f;
+  for (int r0 = 0; r0 < R; r0 += kGateR) {
+    const int rn = min(kGateR, R - r0);
+    __syncthreads();
+    // stage V rows r = g*d + c in [r0, r0 + rn), positions p0..p0+31: lanes run over positions,
+    // each loading 8 consecutive channels, so the transposed stores are conflict-free
+    for (int e = tid; e < kGateP * (rn / 8); e += kGateThreads) {
+      const int p = e % kGateP, o = e / kGateP;
+      const int r = r0 + o * 8, g = r / d, c = r % d;
+      const int pos = p0 + p;
+      float v8[8];
+      if (pos < N) load8_as_f32(V + ((size_t)(b * Hkv + g) * N + pos) * d + c, v8);
+      else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v8[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Vt[(o * 8 + i) * kGateP + p] = v8[i];
     }
-    for (int e = tid; e < d * H_pad; e += nth) {
-      int c = e / H_pad, h = e % H_pad;
-      Ds[e] = h < H ? load_as_f32(Delta + (size_t)(g * d + c) * H + h) : 0.f;
+    for (int e = tid; e < rn * HP; e += kGateThreads) {
+      const int rr = e / HP, h = e % HP;
+      Ds[e] = h < H ? load_as_f32(Delta + (size_t)(r0 + rr) * H + h) : 0.f;
     }
     __syncthreads();
-    for (int c = 0; c < d; ++c) {
-      float4 v4 = *reinterpret_cast<const float4*>(Vs + c * kGatePT + tp * 4);
-      float4 d4 = *reinterpret_cast<const float4*>(Ds + c * H_pad + th * 4);
-      float vv[4] = {v4.x, v4.y, v4.z, v4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+    for (int rr = kg; rr < rn; rr += 8) {
+      const float4 v4 = *reinterpret_cast<const float4*>(Vt + rr * kGateP + pg * 4);
+      const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+      float dd[HPT];
+      if constexpr (HPT % 4 == 0) {
+#pragma unroll
+        for (int j = 0; j < HPT; j += 4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(Ds + rr * HP + hg * HPT + j);
+          dd[j] = d4.x; dd[j + 1] = d4.y; dd[j + 2] = d4.z; dd[j + 3] = d4.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < HPT; ++j) dd[j] = Ds[rr * HP + hg * HPT + j];
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(vv[i], dd[j], acc[i][j]);
+        for (int j = 0; j < HPT; ++j) acc[i][j] = fmaf(vv[i], dd[j], acc[i][j]);
     }
-    __syncthreads();
   }
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int h = th * 4 + j;
-    if (h >= H) continue;
-    const float a = A[h];
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int pos = p0 + tp * 4 + i;
-      if (pos >= N) continue;
-      const float x = acc[i][j];
-      const size_t o = (size_t)(b * H + h) * N + pos;
-      delta[o] = expf(a * softplus_f(x));
-      if (x_save) x_save[o] = x;
-    }
+    for (int j = 0; j < HPT; ++j) red[(kg * kGateP + pg * 4 + i) * HP + hg * HPT + j] = acc[i][j];
+  __syncthreads();
+  for (int o = tid; o < kGateP * HP; o += kGateThreads) {
+    const int p = o / HP, h = o % HP;
+    const int pos = p0 + p;
+    if (h >= H || pos >= N) continue;
+    float x = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x += red[(k * kGateP + p) * HP + h];
+    const size_t off = (size_t)(b * H + h) * N + pos;
+    delta[off] = expf(A[h] * softplus_f(x));
+    if (x_save) x_save[off] = x;
   }
 }
 
@@ -213,27 +257,35 @@ __global__ void gate_bwd_reduce_kernel(const float* __restrict__ part, const flo
   }
 }
 
+template <typename T, int HPT>
+cudaError_t launch_gate_fwd_t(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
+                              float* x_save, cudaStream_t s) {
+  constexpr int HP = 4 * HPT;
+  const int smem = (kGateR * kGateP + kGateR * HP + 8 * kGateP * HP) * (int)sizeof(float);
+  auto k = gate_fwd_kernel<T, HPT>;
+  { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
+  dim3 grid((P.N + kGateP - 1) / kGateP, P.B);
+  k<<<grid, kGateThreads, smem, s>>>((const T*)V, (const T*)Delta, A, delta, x_save, P.H, P.Hkv, P.N, P.d);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_gate_fwd_h(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
+                              float* x_save, cudaStream_t s) {
+  if (P.H <= 4) return launch_gate_fwd_t<T, 1>(P, V, Delta, A, delta, x_save, s);
+  if (P.H <= 8) return launch_gate_fwd_t<T, 2>(P, V, Delta, A, delta, x_save, s);
+  if (P.H <= 16) return launch_gate_fwd_t<T, 4>(P, V, Delta, A, delta, x_save, s);
+  if (P.H <= 32) return launch_gate_fwd_t<T, 8>(P, V, Delta, A, delta, x_save, s);
+  if (P.H <= 64) return launch_gate_fwd_t<T, 16>(P, V, Delta, A, delta, x_save, s);
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             float* delta, float* x_save, cudaStream_t s) {
-  const int H_pad = (P.H + 3) / 4 * 4;
-  const int threads = 16 * (H_pad / 4);
-  if (threads > 1024) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)(P.d * kGatePT + P.d * H_pad) * sizeof(float);
-  dim3 grid((P.N + kGatePT - 1) / kGatePT, P.B);
-  if (P.bf16) {
-    auto k = gate_fwd_kernel<uint16_t>;
-    { cudaError_t ea = ensure_smem_limit(k, (int)smem); if (ea != cudaSuccess) return ea; }
-    k<<<grid, threads, smem, s>>>((const uint16_t*)V, (const uint16_t*)Delta, A, delta, x_save, P.H,
-                                  P.Hkv, P.N, P.d, H_pad);
-  } else {
-    auto k = gate_fwd_kernel<float>;
-    { cudaError_t ea = ensure_smem_limit(k, (int)smem); if (ea != cudaSuccess) return ea; }
-    k<<<grid, threads, smem, s>>>((const float*)V, (const float*)Delta, A, delta, x_save, P.H, P.Hkv,
-                                  P.N, P.d, H_pad);
-  }
-  return cudaGetLastError();
+  return P.bf16 ? launch_gate_fwd_h<uint16_t>(P, V, Delta, A, delta, x_save, s)
+                : launch_gate_fwd_h<float>(P, V, Delta, A, delta, x_save, s);
 }
 
 cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t s) {
