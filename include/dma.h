@@ -201,6 +201,28 @@ dma_status_t dma_gate_bwd(const dma_params_t* p, const void* V, const void* Delt
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Gate backward without a workspace, for callers that cannot allocate device memory: code that
+ * runs where it may not call cudaMalloc (for example inside a host application or framework that
+ * owns the GPU's allocator, or a plugin called from another runtime's graph).  The page has no
+ * counterpart of this entry point; it exists for those callers only.
+ *
+ * Arguments and results are those of dma_gate_bwd (outputs within the same tolerance), except
+ * that there is no workspace: the scratch (gx and the partial sums of dA and dDelta, about
+ * 4 * (B*H*N + ceil(N/512)*B*Hkv*d*H) bytes) lives in a fixed array of DMA_NOALLOC_SCRATCH_BYTES
+ * that the library reserves on every GPU that loads it, until the process exits.  A problem whose
+ * scratch does not fit returns DMA_ERR_UNSUPPORTED before anything is launched.  The first call
+ * on a device looks the array's device address up (cudaGetSymbolAddress) with that device
+ * current, so make that first call before any stream capture.  All calls share the one array:
+ * calls whose GPU work overlaps (on different streams or from different host threads on one
+ * device) race on it, so the caller must serialise them.  Nothing is allocated or freed.
+ */
+#define DMA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+dma_status_t dma_gate_bwd_noalloc(const dma_params_t* p, const void* V, const void* Delta,
+                                  const float* A, const float* x_save, const float* delta,
+                                  const float* d_delta, float* dDelta, float* dA, float* dV_gate,
+                                  void* stream);
+
+/*
  * Reads the device status word of `workspace` (synchronises `stream`).  Returns DMA_OK or
  * DMA_ERR_TIMEOUT when a kernel's bounded wait gave up; *code receives the raw word.
  * dma_clear_device_status resets it (asynchronously on `stream`).

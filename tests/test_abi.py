@@ -136,6 +136,10 @@ assert len(args_bad) == 15
 assert lib.dma_attn_bwd(pp, *args_bad) == INVALID
 # gate_bwd(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, ws, ws_bytes, stream)
 assert lib.dma_gate_bwd(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
+# gate_bwd_noalloc(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, stream)
+assert lib.dma_gate_bwd_noalloc(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == INVALID
+pdec = dma.make_params(8, 32, 8, 65536, 128, 2048, Nq=1)   # 64 MiB of gx alone: more than the fixed array
+assert lib.dma_gate_bwd_noalloc(ctypes.byref(pdec), *([FAKE] * 9), None) == UNSUPPORTED
 print("ok")
 """
 

@@ -19,7 +19,7 @@ from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DmaError, DmaParams, DmaWsLayout,
 __all__ = [
     "BLOCK_Q", "DMA_BF16", "DMA_F32", "DmaError", "DmaParams", "LIB_PATH", "load", "exported_names",
     "make_params", "workspace_size", "workspace_layout", "gate", "topk_mask", "attn_fwd", "attn_bwd",
-    "gate_bwd", "check_device_status", "clear_device_status", "abi_version", "alloc_workspace", "forward",
+    "gate_bwd", "gate_bwd_noalloc", "check_device_status", "clear_device_status", "abi_version", "alloc_workspace", "forward",
     "backward",
 ]
 
@@ -100,6 +100,15 @@ def gate_bwd(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, worksp
                                               _ptr(x_save), _ptr(delta), _ptr(d_delta), _ptr(dDelta),
                                               _ptr(dA), _ptr(dV_gate), _ptr(workspace), _nbytes(workspace),
                                               _stream(stream)))
+
+
+def gate_bwd_noalloc(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, stream=None):
+    """dma_gate_bwd without a workspace, for callers that may not allocate device
+    memory; its scratch is a fixed array inside the library (see include/dma.h)."""
+    check("dma_gate_bwd_noalloc", load().dma_gate_bwd_noalloc(ctypes.byref(p), _ptr(V), _ptr(Delta), _ptr(A),
+                                                              _ptr(x_save), _ptr(delta), _ptr(d_delta),
+                                                              _ptr(dDelta), _ptr(dA), _ptr(dV_gate),
+                                                              _stream(stream)))
 
 
 def check_device_status(p, workspace, stream=None) -> int:

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "DMA_OK", 1: "DMA_ERR_INVALID_ARG", 2: "DMA_ERR_UNSUPPORTED",
 DMA_BF16 = 0
 DMA_F32 = 1
 BLOCK_Q = 128
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class DmaParams(ctypes.Structure):
@@ -49,6 +50,8 @@ _SIGS = {
                      c_vp, c_vp, c_vp, c_vp, c_vp, c_vp],
     "dma_gate_bwd": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                      c_vp, c_sz, c_vp],
+    "dma_gate_bwd_noalloc": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                             c_vp],
     "dma_check_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp, ctypes.POINTER(c_i32)],
     "dma_clear_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp],
 }
