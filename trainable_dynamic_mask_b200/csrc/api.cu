@@ -94,6 +94,9 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_counts = take(BH * R.n_blocks * 2 * sizeof(int32_t));
     R.off_lists = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
+    R.off_tw_p = take(BH * R.N * sizeof(int32_t));
+    R.off_tw_rank = take(BH * R.N * sizeof(int32_t));
+    R.off_tw_T = take(BH * (R.n_blocks + 1) * sizeof(int32_t));
   } else {
     R.off_sel = take(BH * R.sel_len * sizeof(int32_t));
     R.off_dec_part = take(BH * R.n_split * (size_t)(R.d + 2) * sizeof(float));

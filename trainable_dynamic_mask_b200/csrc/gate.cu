@@ -66,24 +66,39 @@ gate_fwd_kernel(const T* __restrict__ V, const T* __restrict__ Delta, const floa
     const int rn = min(kGateR, R - r0);
     __syncthreads();
     // stage V rows r = g*d + c in [r0, r0 + rn), positions p0..p0+31: lanes run over positions,
-    // each loading 8 consecutive channels, so the transposed stores are conflict-free
-    for (int e = tid; e < kGateP * (rn / 8); e += kGateThreads) {
+    // each loading 8 consecutive channels, so the transposed stores are conflict-free.  All loads
+    // of a thread are issued before any store so that their latencies overlap.
+    constexpr int kVLoads = kGateP * (kGateR / 8) / kGateThreads;   // 4
+    float v8[kVLoads][8];
+#pragma unroll
+    for (int u = 0; u < kVLoads; ++u) {
+      const int e = tid + u * kGateThreads;
       const int p = e % kGateP, o = e / kGateP;
       const int r = r0 + o * 8, g = r / d, c = r % d;
       const int pos = p0 + p;
-      float v8[8];
-      if (pos < N) load8_as_f32(V + ((size_t)(b * Hkv + g) * N + pos) * d + c, v8);
+      if (o * 8 < rn && pos < N) load8_as_f32(V + ((size_t)(b * Hkv + g) * N + pos) * d + c, v8[u]);
       else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v8[i] = 0.f;
+        for (int i = 0; i < 8; ++i) v8[u][i] = 0.f;
       }
+    }
+    constexpr int kDLoads = kGateR * HP / kGateThreads;   // HP
+    float dl[kDLoads];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) Vt[(o * 8 + i) * kGateP + p] = v8[i];
-    }
-    for (int e = tid; e < rn * HP; e += kGateThreads) {
+    for (int u = 0; u < kDLoads; ++u) {
+      const int e = tid + u * kGateThreads;
       const int rr = e / HP, h = e % HP;
-      Ds[e] = h < H ? load_as_f32(Delta + (size_t)(r0 + rr) * H + h) : 0.f;
+      dl[u] = (rr < rn && h < H) ? load_as_f32(Delta + (size_t)(r0 + rr) * H + h) : 0.f;
     }
+#pragma unroll
+    for (int u = 0; u < kVLoads; ++u) {
+      const int e = tid + u * kGateThreads;
+      const int p = e % kGateP, o = e / kGateP;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Vt[(o * 8 + i) * kGateP + p] = v8[u][i];
+    }
+#pragma unroll
+    for (int u = 0; u < kDLoads; ++u) Ds[tid + u * kGateThreads] = dl[u];
     __syncthreads();
     for (int rr = kg; rr < rn; rr += 8) {
       const float4 v4 = *reinterpret_cast<const float4*>(Vt + rr * kGateP + pg * 4);

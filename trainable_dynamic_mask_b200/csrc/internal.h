@@ -32,6 +32,8 @@ struct Plan {
   size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
   size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
+  size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
+  size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
   size_t off_gx;                       // gate backward: gx [B, H, N] f32
   size_t off_dA_part;                  // gate backward: [B*H][ceil(N/1024)] f32
   size_t off_dDelta_part;              // gate backward: [n_slices*B][Hkv*d][H] f32

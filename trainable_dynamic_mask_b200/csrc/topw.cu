@@ -30,8 +30,6 @@ namespace dma {
 namespace {
 
 constexpr int kC = kBlockQ;         // chunk = query block = 128
-constexpr int kSortWarps = 16;
-constexpr int kSortThreads = kSortWarps * 32;
 
 DMA_DEVINL uint32_t lanemask_lt() {
   uint32_t m;
@@ -45,151 +43,170 @@ DMA_DEVINL int nth_set_bit(uint32_t x, int n) {
   return __ffs(x) - 1;
 }
 
-struct TopwSmem {
-  uint32_t* keyA;   // [N]   (later: count table, shared with keyB)
-  uint32_t* keyB;   // [N]
-  uint16_t* idxA;   // [N]   after sorting: p[r]
-  uint16_t* idxB;   // [N]   after sorting: rank[j]
-  uint32_t* hist;   // [256 * kSortWarps]
-  int32_t* T;       // [nch + 1]
-  uint16_t* cand;   // [kSortWarps][kC]
-  int32_t* scan;    // [kSortThreads]
-};
+// ---------------------------------------------------------------- sort + thresholds (per row)
 
-__global__ void __launch_bounds__(kSortThreads, 1)
-topw_rows_kernel(const float* __restrict__ delta, int32_t* __restrict__ evict,
-                 int32_t* __restrict__ status, int N, int w) {
+constexpr int kSortThreads2 = 1024;
+constexpr int kSortWarps2 = kSortThreads2 / 32;
+constexpr int kMaxItems = kTopwMaxN / kSortThreads2;   // 16 keys per thread at most
+
+// Shared-memory index with one pad word every 32: thread t's run [IT*t, IT*t + IT) starts in a
+// different bank for every lane of a warp when IT is a power of two.
+DMA_DEVINL int pad32(int i) { return i + (i >> 5); }
+
+// One CTA per (b, h) row: stable LSD radix sort of the row by (delta descending, index ascending)
+// with 4-bit digits, thread-private digit counters and a block-wide scan per pass (digit positions
+// where every key agrees are skipped); then the threshold ranks T_k for every chunk boundary.
+// Writes p (rank -> position), rank (position -> rank) and T to global scratch.
+__global__ void __launch_bounds__(kSortThreads2, 1)
+topw_sort_kernel(const float* __restrict__ delta, int32_t* __restrict__ p_out, int32_t* __restrict__ rank_out,
+                 int32_t* __restrict__ T_out, int N, int w) {
   extern __shared__ __align__(16) unsigned char smraw[];
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = (N + kC - 1) / kC;
-  const int Nal = (N + 7) & ~7;
-  TopwSmem S;
-  S.keyA = reinterpret_cast<uint32_t*>(smraw);
-  S.keyB = S.keyA + Nal;
-  S.idxA = reinterpret_cast<uint16_t*>(S.keyB + Nal);
-  S.idxB = S.idxA + Nal;
-  S.hist = reinterpret_cast<uint32_t*>(S.idxB + Nal);
-  S.T = reinterpret_cast<int32_t*>(S.hist + 256 * kSortWarps);
-  S.cand = reinterpret_cast<uint16_t*>(S.T + ((nch + 1 + 3) & ~3));
-  S.scan = reinterpret_cast<int32_t*>(S.cand + kSortWarps * kC);
+  const int Np = pad32(N) + 32;
+  const int Npi = (Np + 7) & ~7;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smraw);                         // [Np]   (later: table)
+  uint16_t* idx = reinterpret_cast<uint16_t*>(keys + Np);                      // [Npi]  ping
+  uint16_t* idx2 = idx + Npi;                                                  // [Npi]  pong
+  uint16_t* cnt = idx2 + Npi;                                                  // [16][1024] (later: rank)
+  int32_t* wsum = reinterpret_cast<int32_t*>(cnt + 16 * kSortThreads2);        // [32]
+  int32_t* Tsm = wsum + 32;                                                    // [nch + 1]
+  __shared__ uint32_t red_and[kSortWarps2], red_or[kSortWarps2];
 
   const float* drow = delta + (size_t)row * N;
-  int32_t* erow = evict + (size_t)row * N;
-
-  // ---- 1. stable radix sort, ascending on ~order_key (= delta descending, index ascending)
-  for (int i = tid; i < N; i += kSortThreads) {
-    S.keyA[i] = ~order_key(drow[i]);
-    S.idxA[i] = (uint16_t)i;
-  }
-  const int seg = ((N + kSortWarps - 1) / kSortWarps + 31) & ~31;
-  const int wbeg = warp * seg, wend = min(N, wbeg + seg);
-  uint32_t* kin = S.keyA;
-  uint32_t* kout = S.keyB;
-  uint16_t* iin = S.idxA;
-  uint16_t* iout = S.idxB;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = pass * 8;
-    for (int i = tid; i < 256 * kSortWarps; i += kSortThreads) S.hist[i] = 0;
-    __syncthreads();
-    for (int base = wbeg; base < wend; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < wend;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-      if (valid) {
-        const uint32_t dig = (kin[i] >> shift) & 255u;
-        const uint32_t peers = __match_any_sync(vmask, dig);
-        if (lane == __ffs(peers) - 1) S.hist[dig * kSortWarps + warp] += __popc(peers);
+  const int IT = (N + kSortThreads2 - 1) / kSortThreads2;
+  uint32_t kand = 0xffffffffu, kor = 0u;
+  {
+    float dv[kMaxItems];   // all loads first, then the stores
+#pragma unroll
+    for (int u = 0; u < kMaxItems; ++u) {
+      const int i = tid + u * kSortThreads2;
+      dv[u] = i < N ? drow[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kMaxItems; ++u) {
+      const int i = tid + u * kSortThreads2;
+      if (i < N) {
+        const uint32_t k = ~order_key(dv[u]);   // ascending k = delta descending
+        keys[pad32(i)] = k;
+        idx[pad32(i)] = (uint16_t)i;
+        kand &= k;
+        kor |= k;
       }
-      __syncwarp();
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+  }
+  if (lane == 0) { red_and[warp] = kand; red_or[warp] = kor; }
+  __syncthreads();
+  uint32_t varying = 0;
+  {
+    uint32_t a = 0xffffffffu, o = 0u;
+    for (int i = 0; i < kSortWarps2; ++i) { a &= red_and[i]; o |= red_or[i]; }
+    varying = a ^ o;
+  }
+
+  for (int shift = 0; shift < 32; shift += 4) {
+    if (((varying >> shift) & 0xFu) == 0) continue;   // every key has the same digit here
+    uint32_t kk[kMaxItems];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) cnt[c * kSortThreads2 + tid] = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxItems; ++i) {
+      const int pos = tid * IT + i;
+      if (i < IT && pos < N) {
+        kk[i] = keys[pad32(pos)];
+        const uint32_t dg = (kk[i] >> shift) & 0xFu;
+        cnt[dg * kSortThreads2 + tid] += 1;
+      }
     }
     __syncthreads();
-    {  // exclusive scan of hist in (digit, warp) order: 4096 entries, 8 per thread
-      uint32_t v[8], sum = 0;
+    {  // exclusive scan of cnt in (digit, thread) order: 16 entries per thread
+      uint32_t v[16], sum = 0;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) { v[k] = S.hist[tid * 8 + k]; sum += v[k]; }
+      for (int c = 0; c < 16; ++c) { v[c] = cnt[tid * 16 + c]; sum += v[c]; }
       uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (lane == 31) S.scan[warp] = (int32_t)incl;
+      if (lane == 31) wsum[warp] = (int32_t)incl;
       __syncthreads();
       if (warp == 0) {
-        uint32_t ws = lane < kSortWarps ? (uint32_t)S.scan[lane] : 0u;
-        uint32_t wi = ws;
+        const uint32_t x = (uint32_t)wsum[lane];
+        uint32_t xi = x;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
-          if (lane >= o) wi += y;
+          const uint32_t y = __shfl_up_sync(0xffffffffu, xi, o);
+          if (lane >= o) xi += y;
         }
-        if (lane < kSortWarps) S.scan[lane] = (int32_t)(wi - ws);
+        wsum[lane] = (int32_t)(xi - x);
       }
       __syncthreads();
-      uint32_t run = (uint32_t)S.scan[warp] + incl - sum;
+      uint32_t run = (uint32_t)wsum[warp] + incl - sum;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) { S.hist[tid * 8 + k] = run; run += v[k]; }
+      for (int c = 0; c < 16; ++c) { cnt[tid * 16 + c] = (uint16_t)run; run += v[c]; }
     }
     __syncthreads();
-    for (int base = wbeg; base < wend; base += 32) {
-      const int i = base + lane;
-      const bool valid = i < wend;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, valid);
-      uint32_t key = 0, dig = 0, peers = 0, dst = 0;
-      uint16_t idx = 0;
-      if (valid) {
-        key = kin[i];
-        idx = iin[i];
-        dig = (key >> shift) & 255u;
-        peers = __match_any_sync(vmask, dig);
-        dst = S.hist[dig * kSortWarps + warp] + __popc(peers & lanemask_lt());
+    // every read of `keys` in this pass happened before the barriers above, so items can be
+    // written as soon as their destinations are known; indices go to the other buffer
+#pragma unroll
+    for (int i = 0; i < kMaxItems; ++i) {
+      const int pos = tid * IT + i;
+      if (i < IT && pos < N) {
+        const uint32_t dg = (kk[i] >> shift) & 0xFu;
+        const int dst = cnt[dg * kSortThreads2 + tid];
+        cnt[dg * kSortThreads2 + tid] = (uint16_t)(dst + 1);
+        keys[pad32(dst)] = kk[i];
+        idx2[pad32(dst)] = idx[pad32(pos)];
       }
-      __syncwarp();
-      if (valid) {
-        kout[dst] = key;
-        iout[dst] = idx;
-        if (lane == __ffs(peers) - 1) S.hist[dig * kSortWarps + warp] += __popc(peers);
-      }
-      __syncwarp();
     }
     __syncthreads();
-    uint32_t* tk = kin; kin = kout; kout = tk;
-    uint16_t* ti = iin; iin = iout; iout = ti;
+    uint16_t* t = idx; idx = idx2; idx2 = t;
   }
-  // after 4 passes the sorted order is back in (keyA, idxA)
-  const uint16_t* p = S.idxA;   // p[r]
-  uint16_t* rank = S.idxB;      // rank[j]
-  for (int r = tid; r < N; r += kSortThreads) rank[p[r]] = (uint16_t)r;
-
-  // ---- 2. thresholds T_k, k = 0..nch
-  uint32_t* cnt = S.keyA;   // [nch][nch + 1] (spans keyA and keyB)
+  // p[r] = idx[pad32(r)];  rank[j] in the counter area
+  uint16_t* rank = cnt;
+  int32_t* prow = p_out + (size_t)row * N;
+  int32_t* rrow = rank_out + (size_t)row * N;
+  for (int r = tid; r < N; r += kSortThreads2) {
+    const int j = idx[pad32(r)];
+    rank[j] = (uint16_t)r;
+    prow[r] = j;
+    rrow[j] = r;
+  }
+  // thresholds: table[rb][k] = #positions < k*C whose rank is in bucket rb (u32, reuses keys)
+  uint32_t* table = keys;
   const int cw = nch + 1;
-  for (int i = tid; i < nch * cw; i += kSortThreads) cnt[i] = 0;
+  for (int i = tid; i < nch * cw; i += kSortThreads2) table[i] = 0;
   __syncthreads();
-  for (int j = tid; j < N; j += kSortThreads) atomicAdd(&cnt[(rank[j] >> 7) * cw + (j >> 7)], 1u);
+  for (int j = tid; j < N; j += kSortThreads2) atomicAdd(&table[(rank[j] >> 7) * cw + (j >> 7)], 1u);
   __syncthreads();
-  for (int rb = tid; rb < nch; rb += kSortThreads) {
+  for (int rb = tid; rb < nch; rb += kSortThreads2) {
     uint32_t prev = 0;
     for (int k = 0; k <= nch; ++k) {
-      const uint32_t t = cnt[rb * cw + k];
-      cnt[rb * cw + k] = prev;   // positions < k*C with rank in bucket rb
+      const uint32_t t = table[rb * cw + k];
+      table[rb * cw + k] = prev;
       prev += t;
     }
   }
   __syncthreads();
-  for (int k = warp; k <= nch; k += kSortWarps) {
+  for (int k = warp; k <= nch; k += kSortWarps2) {
     const int Pk = min(k * kC, N);
     int Tk = N;
     if (Pk > w) {
       int before = 0, rbs = -1;
       for (int rb0 = 0; rb0 < nch && rbs < 0; rb0 += 32) {
         const int rb = rb0 + lane;
-        const int v = rb < nch ? (int)cnt[rb * cw + k] : 0;
+        const int v = rb < nch ? (int)table[rb * cw + k] : 0;
         int incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          int y = __shfl_up_sync(0xffffffffu, incl, o);
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += y;
         }
         const uint32_t hit = __ballot_sync(0xffffffffu, before + incl >= w);
@@ -201,85 +218,110 @@ topw_rows_kernel(const float* __restrict__ delta, int32_t* __restrict__ evict,
           before += __shfl_sync(0xffffffffu, incl, 31);
         }
       }
-      int need = w - before;   // >= 1: the need-th present rank in bucket rbs
+      int need = w - before;
       for (int r0 = rbs * 128; r0 < min(rbs * 128 + 128, N); r0 += 32) {
         const int r = r0 + lane;
-        const uint32_t m = __ballot_sync(0xffffffffu, r < N && p[r] < Pk);
+        const uint32_t m = __ballot_sync(0xffffffffu, r < N && (int)idx[pad32(min(r, N - 1))] < Pk);
         const int c = __popc(m);
         if (c >= need) { Tk = r0 + nth_set_bit(m, need - 1); break; }
         need -= c;
       }
     }
-    if (lane == 0) S.T[k] = Tk;
+    if (lane == 0) T_out[(size_t)row * cw + k] = Tk;
+  }
+}
+
+// ---------------------------------------------------------------- eviction index (per chunk)
+
+constexpr int kEvThreads = 128;
+
+// One CTA per (chunk k, row).  Chunk k = positions [t0, t1) resolves exactly the keys evicted
+// inside it: old keys (position < t0) with rank in (T_{k+1}, T_k], and its own keys with rank above
+// T_{k+1}.  For such a key of rank r, e = max(j, first t >= t0 with #{i <= t : rank_i < r} >= w);
+// the count over old positions follows from T_k: Sk - #{old candidates with rank >= r}, Sk being
+// min(t0, w).  Its own keys that survive the last boundary get e = N.
+__global__ void __launch_bounds__(kEvThreads)
+topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in,
+                  const int32_t* __restrict__ T_in, int32_t* __restrict__ evict, int32_t* __restrict__ status,
+                  int N, int w) {
+  __shared__ int32_t crank[kC];      // ranks of the chunk's own keys
+  __shared__ int32_t L[kC];          // old candidates, ascending rank
+  __shared__ int32_t wcount[kEvThreads / 32];
+  __shared__ int32_t nL_sh;
+  const int k = blockIdx.x, row = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nch = (N + kC - 1) / kC;
+  const int t0 = k * kC, t1 = min(t0 + kC, N);
+  const int32_t* prow = p_in + (size_t)row * N;
+  const int32_t* rrow = rank_in + (size_t)row * N;
+  const int32_t* T = T_in + (size_t)row * (nch + 1);
+  int32_t* erow = evict + (size_t)row * N;
+  const int Ta = T[k], Tb = T[k + 1], Tf = T[nch];
+  const int Sk = min(t0, w);
+  if (tid < t1 - t0) crank[tid] = rrow[t0 + tid];
+  // old candidates in rank order
+  int nL = 0;
+  const int rhi = min(Ta, N - 1);
+  for (int r0 = Tb + 1; r0 <= rhi; r0 += kEvThreads) {
+    const int r = r0 + tid;
+    const bool in = r <= rhi && prow[r] < t0;
+    const uint32_t m = __ballot_sync(0xffffffffu, in);
+    if (lane == 0) wcount[warp] = __popc(m);
+    __syncthreads();
+    int before = nL, total = 0;
+    for (int i = 0; i < kEvThreads / 32; ++i) {
+      if (i < warp) before += wcount[i];
+      total += wcount[i];
+    }
+    if (in) {
+      const int slot = before + __popc(m & lanemask_lt());
+      if (slot < kC) L[slot] = r;
+    }
+    nL += total;
+    __syncthreads();
+  }
+  if (nL > kC) {   // cannot happen: at most C keys are evicted per chunk
+    if (tid == 0) atomicOr(status, 2);
+    nL = kC;
   }
   __syncthreads();
-
-  // ---- 3. eviction index, chunk by chunk
-  const int Tf = S.T[nch];
-  uint16_t* L = S.cand + warp * kC;
-  for (int k = warp; k < nch; k += kSortWarps) {
-    const int t0 = k * kC, t1 = min(t0 + kC, N);
-    const int Ta = S.T[k], Tb = S.T[k + 1];
-    const int Sk = min(t0, w);
-    // old candidates: rank in (Tb, min(Ta, N-1)] and position < t0, ascending rank
-    int nL = 0;
-    const int rhi = min(Ta, N - 1);
-    for (int r0 = Tb + 1; r0 <= rhi; r0 += 32) {
-      const int r = r0 + lane;
-      const bool in = r <= rhi && p[r] < t0;
-      const uint32_t m = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const int slot = nL + __popc(m & lanemask_lt());
-        if (slot < kC) L[slot] = (uint16_t)r;
+  const int ncand = nL + (t1 - t0);
+  for (int c = tid; c < ncand; c += kEvThreads) {
+    int r, j, base, e = -1;
+    bool scan = false;
+    if (c < nL) {
+      r = L[c];
+      j = prow[r];
+      base = Sk - (nL - c);
+      scan = true;
+    } else {
+      j = t0 + (c - nL);
+      r = crank[c - nL];
+      base = 0;
+      if (r <= Tb) {
+        if (r <= Tf) e = N;            // never evicted
+      } else if (Ta < N && r > Ta) {
+        e = j;                         // never selected
+      } else {
+        int above = 0;                 // old members with rank in (r, Ta]
+        for (int i = 0; i < nL; ++i) above += L[i] > r;
+        base = Sk - above;
+        if (base >= w) e = j;
+        else scan = true;
       }
-      nL += __popc(m);
     }
-    if (nL > kC) {   // cannot happen: at most C keys are evicted per chunk
-      if (lane == 0) atomicOr(status, 2);
-      nL = kC;
-    }
-    __syncwarp();
-    // candidates: old (index < nL) then new (positions t0..t1-1)
-    const int ncand = nL + (t1 - t0);
-    for (int c0 = 0; c0 < ncand; c0 += 32) {
-      const int c = c0 + lane;
-      int r = 0, j = 0, base = 0, e = -1;
-      bool scan = false;
-      if (c < nL) {
-        r = L[c];
-        j = p[r];
-        base = Sk - (nL - c);
-        scan = true;
-      } else if (c < ncand) {
-        j = t0 + (c - nL);
-        r = rank[j];
-        if (r <= Tb) {
-          if (r <= Tf) e = N;          // never evicted
-        } else if (Ta < N && r > Ta) {
-          e = j;                       // never selected
-        } else {
-          int above = 0;               // old members with rank in (r, Ta]
-          for (int i = 0; i < nL; ++i) above += (int)L[i] > r;
-          base = Sk - above;
-          if (base >= w) e = j;
-          else scan = true;
-        }
-      }
-      bool active = scan;
+    if (scan) {
       int count = base;
-      for (int t = t0; t < t1 && __any_sync(0xffffffffu, active); ++t) {
-        const int rt = rank[t];
-        if (active && rt < r) {
-          if (++count >= w) { e = max(j, t); active = false; }
-        }
+      e = -2;
+      for (int t = t0; t < t1; ++t) {
+        if (crank[t - t0] < r && ++count >= w) { e = max(j, t); break; }
       }
-      if (active) {   // cannot happen: such keys are evicted inside the chunk
+      if (e == -2) {                   // cannot happen: such keys are evicted inside the chunk
         e = t1;
         atomicOr(status, 4);
       }
-      if (c < ncand && e >= 0) erow[j] = e;
     }
-    __syncwarp();
+    if (e >= 0) erow[j] = e;
   }
 }
 
@@ -297,13 +339,25 @@ topw_lists_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ count
   const int32_t* erow = evict + (size_t)row * N;
   int32_t* out = lists + ((size_t)row * n_blocks + k) * list_cap;
   int nfull = 0, npart = 0;
+  int enext[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int j = tid * 4 + u;
+    enext[u] = j < t1 ? erow[j] : 0;
+  }
   for (int base = 0; base < t1; base += kListThreads * 4) {
-    int f[4], q[4];
+    int f[4], q[4], ecur[4];
     int cf = 0, cq = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
+      ecur[u] = enext[u];
+      const int jn = base + kListThreads * 4 + tid * 4 + u;   // prefetch the next round
+      enext[u] = jn < t1 ? erow[jn] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
       const int j = base + tid * 4 + u;
-      int e = j < t1 ? erow[j] : 0;
+      const int e = ecur[u];
       const bool live = j < t1 && e > max(j, t0);
       const bool full = live && j <= t0 && e >= t1;
       f[u] = full;
@@ -449,25 +503,21 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
 
 }  // namespace
 
-size_t topw_rows_smem_bytes(int N) {
-  const int nch = (N + kC - 1) / kC;
-  const size_t Nal = (size_t)((N + 7) & ~7);
-  size_t b = Nal * 4 * 2 + Nal * 2 * 2 + 256 * kSortWarps * 4 + (size_t)((nch + 1 + 3) & ~3) * 4 +
-             kSortWarps * kC * 2 + kSortThreads * 4;
-  // the count table [nch][nch+1] u32 reuses keyA+keyB
-  const size_t table = (size_t)nch * (nch + 1) * 4;
-  if (table > Nal * 8) b += table - Nal * 8;   // only for tiny N
-  return b;
-}
-
 cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evict, void* ws,
                                 cudaStream_t s) {
   const int rows = P.B * P.H;
-  size_t smem = topw_rows_smem_bytes(P.N);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  { cudaError_t ea = ensure_smem_limit(topw_rows_kernel, (int)smem); if (ea != cudaSuccess) return ea; }
-  topw_rows_kernel<<<rows, kSortThreads, smem, s>>>(delta, evict, ws_ptr<int32_t>(ws, P.off_status),
-                                                   P.N, P.w);
+  const int nch = P.n_blocks;
+  const int Np = P.N + (P.N >> 5) + 32;
+  const size_t smem = (size_t)Np * 4 + (size_t)((Np + 7) & ~7) * 2 * 2 + 16 * kSortThreads2 * 2 + 32 * 4 +
+                      (size_t)(nch + 1) * 4;
+  if ((size_t)nch * (nch + 1) * 4 > (size_t)Np * 4) return cudaErrorInvalidValue;   // table must fit
+  { cudaError_t ea = ensure_smem_limit(topw_sort_kernel, (int)smem); if (ea != cudaSuccess) return ea; }
+  int32_t* pbuf = ws_ptr<int32_t>(ws, P.off_tw_p);
+  int32_t* rbuf = ws_ptr<int32_t>(ws, P.off_tw_rank);
+  int32_t* Tbuf = ws_ptr<int32_t>(ws, P.off_tw_T);
+  topw_sort_kernel<<<rows, kSortThreads2, smem, s>>>(delta, pbuf, rbuf, Tbuf, P.N, P.w);
+  topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
+                                                            ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
   topw_lists_kernel<<<dim3(P.n_blocks, rows), kListThreads, 0, s>>>(
       evict, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists), P.N, P.list_cap,
       P.n_blocks);
