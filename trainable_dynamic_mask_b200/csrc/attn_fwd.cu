@@ -416,6 +416,12 @@ cudaError_t launch_dec_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
 cudaError_t launch_attn_fwd(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                             const float* delta, const int32_t* evict, void* ws, void* O, float* LSE,
                             cudaStream_t s) {
+  return launch_attn_fwd_tc(P, Q, K, V, delta, evict, ws, O, LSE, s);
+}
+
+cudaError_t launch_attn_fwd_mma_sync(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                     const float* delta, const int32_t* evict, void* ws, void* O, float* LSE,
+                                     cudaStream_t s) {
   if (P.d == 128)
     return P.bf16 ? launch_fwd_t<128, uint16_t>(P, Q, K, V, delta, evict, ws, O, LSE, s)
                   : launch_fwd_t<128, float>(P, Q, K, V, delta, evict, ws, O, LSE, s);

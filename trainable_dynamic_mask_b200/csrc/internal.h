@@ -56,6 +56,9 @@ cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n
 cudaError_t launch_attn_fwd(const Plan& P, const uint16_t* Q, const uint16_t* K,
                             const uint16_t* V, const float* delta, const int32_t* evict,
                             void* ws, void* O, float* LSE, cudaStream_t s);
+cudaError_t launch_attn_fwd_tc(const Plan& P, const uint16_t* Q, const uint16_t* K,
+                               const uint16_t* V, const float* delta, const int32_t* evict,
+                               void* ws, void* O, float* LSE, cudaStream_t s);
 cudaError_t launch_decode_attn(const Plan& P, const uint16_t* Q, const uint16_t* K,
                                const uint16_t* V, const float* delta, void* ws, void* O,
                                float* LSE, cudaStream_t s);

@@ -71,7 +71,6 @@ topw_sort_kernel(const float* __restrict__ delta, int32_t* __restrict__ p_out, i
   uint16_t* idx2 = idx + Npi;                                                  // [Npi]  pong
   uint16_t* cnt = idx2 + Npi;                                                  // [16][1024] (later: rank)
   int32_t* wsum = reinterpret_cast<int32_t*>(cnt + 16 * kSortThreads2);        // [32]
-  int32_t* Tsm = wsum + 32;                                                    // [nch + 1]
   __shared__ uint32_t red_and[kSortWarps2], red_or[kSortWarps2];
 
   const float* drow = delta + (size_t)row * N;
@@ -247,7 +246,6 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   __shared__ int32_t crank[kC];      // ranks of the chunk's own keys
   __shared__ int32_t L[kC];          // old candidates, ascending rank
   __shared__ int32_t wcount[kEvThreads / 32];
-  __shared__ int32_t nL_sh;
   const int k = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = (N + kC - 1) / kC;
