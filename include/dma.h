@@ -155,7 +155,9 @@ dma_status_t dma_gate(const dma_params_t* p, const void* V, const void* Delta, c
  *          j is no longer among the w best causal keys (N if never).  Query t selects key j
  *          iff j <= t < e_j; e_j == j means key j is never selected.  Because delta does not
  *          depend on the query, the queries selecting a key always form this interval.
- *          Also writes the per-block live-key lists and counts into the workspace.
+ *          Also writes the per-block live-key lists and counts into the workspace, and beside
+          each list entry the values the attention forward needs for that key (e_j and delta_j),
+          so that its load stage reads them with contiguous loads instead of a gather.
  *          Decode (Nq == 1): `evict` must be NULL; the selected keys of the query at
  *          position N-1 are written to the workspace region off_sel.
  */
@@ -167,7 +169,9 @@ dma_status_t dma_topk_mask(const dma_params_t* p, const float* delta, int32_t* e
  * (masked pairs are skipped, section "Theoretical Guarantees for Safe Computation Skipping").
  *   Q      [B, H, Nq, d] dtype;  K, V [B, Hkv, N, d] dtype;  delta [B, H, N] float32
  *   evict  [B, H, N] int32 from dma_topk_mask (NULL for decode); the workspace must hold the
- *          lists (or selection) dma_topk_mask wrote for the same delta.
+ *          lists (or selection) dma_topk_mask wrote for the same delta.  Prefill takes delta_j
+ *          and e_j from the per-entry copies dma_topk_mask stored with the lists, so a delta
+ *          changed after dma_topk_mask is not seen there: run dma_topk_mask again.
  *   O      [B, H, Nq, d] dtype out;  LSE [B, H, Nq] float32 out
  */
 dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, const void* V,

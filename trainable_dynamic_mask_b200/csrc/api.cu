@@ -93,6 +93,8 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   if (!R.decode) {
     R.off_counts = take(BH * R.n_blocks * 2 * sizeof(int32_t));
     R.off_lists = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
+    R.off_list_je = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
+    R.off_list_dl = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(float));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));

@@ -116,9 +116,9 @@ template <int R> DMA_DEVINL void regs_dec() { asm volatile("setmaxnreg.dec.sync.
 template <int D, typename OutT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const float* __restrict__ delta,
-                   const int32_t* __restrict__ evict, const int32_t* __restrict__ counts,
-                   const int32_t* __restrict__ lists, OutT* __restrict__ O, float* __restrict__ LSE,
+                   const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ counts, const int32_t* __restrict__ lists,
+                   const int32_t* __restrict__ list_je, const float* __restrict__ list_dl,
+                   OutT* __restrict__ O, float* __restrict__ LSE,
                    int32_t* __restrict__ status, int H, int G, int N, int n_blocks, int list_cap,
                    float scale_log2) {
   using S = TcSmem<D>;
@@ -174,9 +174,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     const int pw = warp - kProdWarp0;            // producer warp 0..3
     const int prow = pw * 32 + lane;             // the tile row this thread owns
     const int kvrow0 = (b * Hkv + g) * N;
-    const float* drow = delta + (size_t)bh * N;
-    const int32_t* erow = evict + (size_t)bh * N;
-    const int32_t* list = lists + ((size_t)bh * n_blocks + kb) * list_cap;
+    const size_t lbase = ((size_t)bh * n_blocks + kb) * list_cap;
+    const int32_t* list = lists + lbase;
+    const int32_t* lje = list_je + lbase;
+    const float* ldl = list_dl + lbase;
     constexpr uint32_t kRowBytes = D * 2;
     const bool issuer = lane < 8;                // lanes 0-7 gather rows pw*32 + 4*lane .. +3
     const uint32_t goff = (uint32_t)(pw * 32 + 4 * (lane & 7)) * 128;
@@ -189,26 +190,27 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       for (int hf = 0; hf < D / 64; ++hf)
         tma_gather4(smem_u32(sm + S::kQ) + hf * 16384 + goff, &qmap, hf * 64, r[0], r[1], r[2], r[3], &bar.q_full);
     }
-    // Software pipeline over tiles: this row's list entry is loaded two tiles ahead and its delta,
-    // e one tile ahead, so that global-load latencies overlap the waits for free stages.
-    auto list_at = [&](int i) {
+    // Software pipeline over tiles: this row's list entry and its metadata (written beside the list
+    // by the list kernel, so no load depends on another) are loaded two tiles ahead.
+    struct Entry { int j, je; float dl; };
+    auto entry_at = [&](int i) {
       const int li = i * kTcBK + prow;
-      return (i < n_tiles && li < n_live) ? list[li] : -1;
+      Entry x{-1, 0xffff, 0.f};
+      if (i < n_tiles && li < n_live) { x.j = list[li]; x.je = lje[li]; x.dl = ldl[li]; }
+      return x;
     };
-    int jc = list_at(0), jn = list_at(1), jv = -1;
-    float dc = jc >= 0 ? drow[jc] : 0.f;
-    int ec = jc >= 0 ? erow[jc] : 0;
+    Entry ec = entry_at(0), en = entry_at(1);
+    int jv = -1;
     for (int i = 0; run && i <= n_tiles; ++i) {
-      const int jnn = list_at(i + 2);
-      const float dn = (i + 1 < n_tiles && jn >= 0) ? drow[jn] : 0.f;
-      const int en = (i + 1 < n_tiles && jn >= 0) ? erow[jn] : 0;
+      const Entry enn = entry_at(i + 2);
+      const int jc = ec.j;
       if (i < n_tiles) {
         const int ks = i % kKStages, ms = i % kMStages;
         if (i >= kMStages &&
             !wait_all(&bar.m_empty[ms], ((i / kMStages) - 1) & 1, abort_flag, status, kErrTimeoutMEmpty))
           break;
-        m_dl[ms * kTcBK + prow] = dc * kLog2e;
-        m_je[ms * kTcBK + prow] = (jc & 0xffff) | (ec << 16);
+        m_dl[ms * kTcBK + prow] = ec.dl;
+        m_je[ms * kTcBK + prow] = ec.je;
         tc::mbar_arrive(&bar.m_full[ms]);
         if (i >= kKStages &&
             !wait_all(&bar.k_empty[ks], ((i / kKStages) - 1) & 1, abort_flag, status, kErrTimeoutKEmpty))
@@ -248,10 +250,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
       }
       jv = jc;
-      jc = jn;
-      jn = jnn;
-      dc = dn;
       ec = en;
+      en = enn;
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -511,8 +511,12 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
   const int smem = TcSmem<D>::kBytes;
   { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
   dim3 grid(P.n_blocks, P.B * P.H);
-  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, delta, evict, ws_ptr<int32_t>(ws, P.off_counts),
-                                   ws_ptr<int32_t>(ws, P.off_lists), (OutT*)O, LSE,
+  // delta and e enter through the per-entry metadata that the list kernel wrote beside the lists
+  (void)delta;
+  (void)evict;
+  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
+                                   ws_ptr<int32_t>(ws, P.off_list_je), ws_ptr<float>(ws, P.off_list_dl),
+                                   (OutT*)O, LSE,
                                    ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_blocks, P.list_cap,
                                    P.scale * kLog2e);
   return cudaGetLastError();

@@ -34,6 +34,7 @@ struct Plan {
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
   size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
+  size_t off_list_je, off_list_dl;     // per list entry: j | e_j << 16 (i32), delta_j * log2(e) (f32)
   size_t off_gx;                       // gate backward: gx [B, H, N] f32
   size_t off_dA_part;                  // gate backward: [B*H][ceil(N/1024)] f32
   size_t off_dDelta_part;              // gate backward: [n_slices*B][Hkv*d][H] f32

@@ -327,15 +327,20 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
 constexpr int kListThreads = 256;
 
 __global__ void __launch_bounds__(kListThreads)
-topw_lists_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ counts,
-                  int32_t* __restrict__ lists, int N, int list_cap, int n_blocks) {
+topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
+                  int32_t* __restrict__ counts, int32_t* __restrict__ lists, int32_t* __restrict__ list_je,
+                  float* __restrict__ list_dl, int N, int list_cap, int n_blocks) {
   __shared__ int32_t partial[2 * kC];
   __shared__ int32_t wsum[2][kListThreads / 32];
   const int k = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = k * kC, t1 = min(t0 + kC, N);
   const int32_t* erow = evict + (size_t)row * N;
-  int32_t* out = lists + ((size_t)row * n_blocks + k) * list_cap;
+  const size_t lbase = ((size_t)row * n_blocks + k) * list_cap;
+  int32_t* out = lists + lbase;
+  int32_t* oje = list_je + lbase;   // j | e_j << 16 of each entry (what the attention kernel tests)
+  float* odl = list_dl + lbase;     // delta_j * log2(e)
+  const float* drow = delta + (size_t)row * N;
   int nfull = 0, npart = 0;
   int enext[4];
 #pragma unroll
@@ -382,7 +387,14 @@ topw_lists_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ count
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = base + tid * 4 + u;
-      if (f[u]) { if (of < list_cap) out[of] = j; ++of; }
+      if (f[u]) {
+        if (of < list_cap) {
+          out[of] = j;
+          oje[of] = (j & 0xffff) | (ecur[u] << 16);
+          odl[of] = drow[j] * kLog2e;
+        }
+        ++of;
+      }
       if (q[u]) { if (oq < 2 * kC) partial[oq] = j; ++oq; }
     }
     nfull += tf;
@@ -392,7 +404,20 @@ topw_lists_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ count
   // at most C evicted old keys plus C new keys; a live set never exceeds list_cap
   nfull = min(nfull, list_cap);
   npart = min(min(npart, 2 * kC), list_cap - nfull);
-  for (int i = tid; i < npart; i += kListThreads) out[nfull + i] = partial[i];
+  for (int i = tid; i < npart; i += kListThreads) {
+    const int j = partial[i];
+    out[nfull + i] = j;
+    oje[nfull + i] = (j & 0xffff) | (erow[j] << 16);
+    odl[nfull + i] = drow[j] * kLog2e;
+  }
+  // pad the last 128-entry tile: key -1 is masked everywhere
+  const int nlive = nfull + npart;
+  const int nround = min(list_cap, (nlive + kC - 1) / kC * kC);
+  for (int i = nlive + tid; i < nround; i += kListThreads) {
+    out[i] = -1;
+    oje[i] = 0xffff;
+    odl[i] = 0.f;
+  }
   if (tid == 0) {
     counts[((size_t)row * n_blocks + k) * 2 + 0] = nfull;
     counts[((size_t)row * n_blocks + k) * 2 + 1] = nfull + npart;
@@ -517,8 +542,8 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
   topw_lists_kernel<<<dim3(P.n_blocks, rows), kListThreads, 0, s>>>(
-      evict, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists), P.N, P.list_cap,
-      P.n_blocks);
+      evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
+      ws_ptr<int32_t>(ws, P.off_list_je), ws_ptr<float>(ws, P.off_list_dl), P.N, P.list_cap, P.n_blocks);
   return cudaGetLastError();
 }
 
