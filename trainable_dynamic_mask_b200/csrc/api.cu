@@ -78,7 +78,11 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     size_t cap = align_up((size_t)minwn + kBlockQ, kBlockQ);
     size_t ncap = align_up((size_t)R.N, kBlockQ);
     R.list_cap = (int)(cap < ncap ? cap : ncap);
+    // a pair's live set: the <= w keys live at its first row plus at most kPairQ new keys
+    size_t pcap = align_up((size_t)minwn + kPairQ, kBlockQ);
+    R.pair_cap = (int)(pcap < ncap ? pcap : ncap);
   }
+  R.n_pairs = (R.N + kPairQ - 1) / kPairQ;
   R.sel_len = minwn;
   R.n_split = (R.sel_len + kDecodeSplit - 1) / kDecodeSplit;
   R.n_slices = (R.N + kGateSlice - 1) / kGateSlice;
@@ -93,8 +97,10 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   if (!R.decode) {
     R.off_counts = take(BH * R.n_blocks * 2 * sizeof(int32_t));
     R.off_lists = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
-    R.off_list_je = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
-    R.off_list_dl = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(float));
+    R.off_pcounts = take(BH * R.n_pairs * 2 * sizeof(int32_t));
+    R.off_plists = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(int32_t));
+    R.off_pje = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(int32_t));
+    R.off_pdl = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(float));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));

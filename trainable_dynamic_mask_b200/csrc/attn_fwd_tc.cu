@@ -5,26 +5,27 @@
 // have weight exactly 0 and are skipped) and "Hardware-Optimized Implementation" (block-wise,
 // FlashAttention-style computation on tensor cores, O(n w d) work).
 //
-// One CTA per (b, h, block of 128 query rows), walking the block's live-key list (full keys first)
-// in tiles of 128 keys.  The tiles are split into two interleaved streams, A (even tiles) and B
-// (odd tiles), each with its own S, P, O and softmax state, so that two softmax warps share every
-// SM sub-partition and the tensor core always has the other stream's work while one stream runs
-// its softmax.  The two partial results are merged at the end.
+// Work item = (b, h, pair of query blocks: 256 rows), walking the pair's live-key list (the union
+// of the two blocks' lists; full keys first) in tiles of 128 keys.  Each gathered K/V tile feeds
+// both 128-row halves, so the gather traffic per tensor-core FLOP is half that of 128-row items.
+// The kernel is persistent: one CTA per SM walks items heaviest-first (snake order over the CTAs),
+// and the next item's Q and first tiles load while the current one finishes.
 //
-// Warp roles (512 threads; warps 9-11 only complete the third warpgroup):
-//   warps 0-3  softmax of stream A, warps 4-7 softmax of stream B: thread r owns query row
-//              r = TMEM lane r.  It reads its S row from TMEM, applies scale, +delta_j and the mask
-//              j <= t < e_j (tiles of full keys skip the test), keeps the running max and sum in
-//              registers, writes P (bf16) back over S in TMEM, and rescales its O row only when the
-//              running max grows by more than 2^8 (the stale max otherwise stays the reference);
-//   warp 8     allocates TMEM; one thread issues the MMAs: S = Q K^T (A and B from shared memory)
-//              and O += P V (A = P from TMEM, B = V from shared memory);
-//   warps 12-15 producers: thread p owns row p of every tile (its list entry, delta*log2(e) and
-//              (j, e_j)); lanes 0-7 of each warp gather 4 rows each of K and V with TMA tile::gather4
-//              (128-byte swizzled, the layout the MMA reads).  The TMA issue rate of one warp caps
-//              gather throughput, so four warps issue.
-// TMEM: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D); P_X aliases S_X.
-// Stages: K 3, V 2 (each stream owns one V stage), metadata 4 (released by the softmax).
+// Warp roles (512 threads):
+//   warps 0-3  softmax of query half 0, warps 4-7 softmax of half 1: thread r owns query row r of
+//              its half = TMEM lane r.  It reads its S row from TMEM, applies scale, +delta_j and the
+//              mask j <= t < e_j (tiles of full keys skip the test), keeps the running max and sum,
+//              writes P (bf16) over S in TMEM, and rescales its O row only when the running max
+//              grows by more than 2^8 (the stale max otherwise stays the reference).  A quarter of
+//              the exponentials run as a polynomial on the FMA pipe to offload the MUFU pipe;
+//   warp 8     allocates TMEM; one thread issues the MMAs: S_h = Q_h K^T (operands in shared
+//              memory) and O_h += P_h V (P_h from TMEM, V from shared memory);
+//   warps 9-11 gather V rows, warps 12-15 gather Q and K rows, with TMA tile::gather4 (128-byte
+//              swizzled, the layout the MMA reads).  One warp's TMA issue rate caps its gather
+//              throughput, so seven warps issue.
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D); P_h aliases S_h.
+// Stages: Q 1 (both halves), K 2, V 2.  Tile metadata (delta_j log2(e), j | e_j << 16) is read by
+// the softmax threads straight from the list, one entry per thread, through a shared buffer.
 // Every wait is bounded (tc::mbar_wait) and reports a timeout through the workspace status word;
 // every TMEM load/store (warp-collective) sits behind warp-uniform decisions.
 #include <cuda.h>
@@ -38,40 +39,40 @@
 namespace dma {
 namespace {
 
-constexpr int kTcThreads = 512;       // 4 warpgroups: softmax A, softmax B, MMA (+3 idle), producers
-constexpr int kProdWarp0 = 12, kProdWarps = 4, kProdThreads = kProdWarps * 32;
-// Register split between the warpgroups (setmaxnreg): launched with 128 per thread (512 x 128 =
-// 65536), the MMA and producer warpgroups give back to 48 and the softmax warpgroups take 208:
-// 256 x 48 + 256 x 208 = 65536, so the increase can always be satisfied.
+constexpr int kTcThreads = 512;
+constexpr int kMmaWarp = 8;
+constexpr int kVWarp0 = 9, kVWarps = 3;     // V producers: row groups 11 + 11 + 10
+constexpr int kKWarp0 = 12, kKWarps = 4;    // Q/K producers: row groups 8 per warp
+// Register split (setmaxnreg): launched with 128 per thread (512 x 128 = 65536), warpgroups 2 and 3
+// give back to 48 and the softmax warpgroups take 208: 256 x 48 + 256 x 208 = 65536.
 constexpr int kRegsSoftmax = 208, kRegsOther = 48;
-constexpr int kTcBK = 128;            // keys per tile
-constexpr int kKStages = 3, kVStages = 2, kMStages = 4;
+constexpr int kTcBK = 128;                  // keys per tile
+constexpr int kKStages = 2, kVStages = 2;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr int kPolyEvery = 4;               // one pair in kPolyEvery takes the polynomial exp2
 
 enum : int { kErrTimeoutQ = 0x100, kErrTimeoutK = 0x200, kErrTimeoutS = 0x400, kErrTimeoutP = 0x800,
              kErrTimeoutPV = 0x1000, kErrTimeoutKEmpty = 0x2000, kErrTimeoutV = 0x4000,
-             kErrTimeoutVEmpty = 0x8000, kErrTimeoutM = 0x10000, kErrTimeoutMEmpty = 0x20000,
-             kErrSmemAlign = 0x40000 };
+             kErrTimeoutVEmpty = 0x8000, kErrTimeoutQEmpty = 0x10000, kErrSmemAlign = 0x40000 };
 
 template <int D>
 struct TcSmem {
   static constexpr int kHalves = D / 64;              // 64-element column halves of a row
   static constexpr int kTile = kHalves * 128 * 128;   // [halves][128 rows][128 B]
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTile;               // [kKStages]
+  static constexpr int kQ = 0;                        // [2 query halves]
+  static constexpr int kK = kQ + 2 * kTile;           // [kKStages]
   static constexpr int kV = kK + kKStages * kTile;    // [kVStages]
-  static constexpr int kMeta = kV + kVStages * kTile; // [kMStages][dl (f32), jj|ee (i32)][128]
-  static constexpr int kMerge = kMeta + kMStages * 2 * kTcBK * 4;   // [2 streams][m, l][128]
-  static constexpr int kBars = kMerge + 2 * 2 * 128 * 4;
+  static constexpr int kMeta = kV + kVStages * kTile; // [2 halves][2 buffers][dl f32 | je i32][128]
+  static constexpr int kBars = kMeta + 2 * 2 * 2 * kTcBK * 4;
   static constexpr int kBytes = kBars + 512;
 };
 
 struct TcBars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t m_full[kMStages], m_empty[kMStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -108,34 +109,159 @@ DMA_DEVINL bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_fla
   return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag, status, code));
 }
 
-DMA_DEVINL void softmax_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+// Wait that ignores the abort flag, for draining copies in flight after an abort (bounded).
+DMA_DEVINL void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!tc::mbar_try_wait(bar, parity) && clock64() - t0 < 200000000LL) {
+  }
+}
+
+// Named barrier of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
+DMA_DEVINL void group_sync(int h) {
+  if (h == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
+  else asm volatile("bar.sync 2, 128;\n" ::: "memory");
+}
 
 template <int R> DMA_DEVINL void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R)); }
 template <int R> DMA_DEVINL void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R)); }
 
+// ---- packed f32x2 arithmetic (two lanes of FP32 work per instruction on sm_100)
+DMA_DEVINL uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+DMA_DEVINL void f2_split(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
+DMA_DEVINL uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+DMA_DEVINL uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+DMA_DEVINL uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+DMA_DEVINL float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of x <= ~8 on the FMA pipe: x = i + f with i = round(x), f in [-1/2, 1/2];
+// 2^f ~ 1 + f (c1 + f (c2 + f c3)), a cubic fitted here for minimum relative error on [-1/2, 1/2]
+// (max 1.02e-4, far below bf16's half ulp 2^-9, the precision P is stored in); i is added to the
+// exponent field.  x is clamped at -127, where f = 0, p = 1 exactly and the exponent sum wraps to
+// +0: masked entries (x = -inf) give exactly 0, as the MUFU path does.  Round-to-nearest uses the
+// 1.5 * 2^23 shift: the integer lands in the low mantissa bits of x + 1.5 * 2^23.
+DMA_DEVINL void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  constexpr float c1 = 0.6932829022407532f, c2 = 0.24221068620681763f, c3 = 0.05500871315598488f;
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  const uint64_t x = f2(x0, x1);
+  const uint64_t r = f2_add(x, f2(kShift, kShift));
+  const uint64_t f = f2_sub(x, f2_sub(r, f2(kShift, kShift)));
+  uint64_t p = f2_fma(f, f2(c3, c3), f2(c2, c2));
+  p = f2_fma(f, p, f2(c1, c1));
+  p = f2_fma(f, p, f2(1.f, 1.f));
+  float r0, r1, q0, q1;
+  f2_split(r, r0, r1);
+  f2_split(p, q0, q1);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
+}
+
+// tcgen05.mma (kind::f16, A and B from shared memory) with both descriptors advanced by OFF / 16
+// inside the asm block: the 8 K steps then need no live descriptor registers each.
+template <uint32_t OFF>
+DMA_DEVINL void mma_ss_at(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
+      "add.s64 a, %1, %5;\n\t"
+      "add.s64 b, %2, %5;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(OFF >> 4));
+}
+// tcgen05.mma with A = P from TMEM column a_tmem + 8 KK and B = V at descriptor + KK * 2048 / 16.
+template <int KK>
+DMA_DEVINL void mma_ts_at(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "add.s64 b, %2, %5;\n\t"
+      "add.u32 a, %1, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(KK * 2048 / 16), "n"(KK * 8));
+}
+
+template <int KK, int NK>
+struct QkSteps {
+  DMA_DEVINL static void run(uint32_t d, uint64_t dq, uint64_t dk, uint32_t id) {
+    mma_ss_at<(KK >> 2) * 16384 + (KK & 3) * 32>(d, dq, dk, id, KK > 0 ? 1u : 0u);
+    QkSteps<KK + 1, NK>::run(d, dq, dk, id);
+  }
+};
+template <int NK>
+struct QkSteps<NK, NK> {
+  DMA_DEVINL static void run(uint32_t, uint64_t, uint64_t, uint32_t) {}
+};
+template <int KK, int NK>
+struct PvSteps {
+  DMA_DEVINL static void run(uint32_t d, uint32_t a, uint64_t dv, uint32_t id, uint32_t acc0) {
+    mma_ts_at<KK>(d, a, dv, id, KK > 0 ? 1u : acc0);
+    PvSteps<KK + 1, NK>::run(d, a, dv, id, acc0);
+  }
+};
+template <int NK>
+struct PvSteps<NK, NK> {
+  DMA_DEVINL static void run(uint32_t, uint32_t, uint64_t, uint32_t, uint32_t) {}
+};
+
+// S_h = Q_h K^T: Q half `half` (descriptor dq0 of half 0), K tile at descriptor dk; commits to `done`.
+// (Shared addresses stay below 2^18, so adding offsets to the 14-bit address field never carries.)
+template <int D>
+DMA_DEVINL void issue_qk(uint32_t tmem, int half, uint64_t dq0, uint64_t dk, uint64_t* done) {
+  constexpr uint32_t idq = tc::idesc_bf16(128, kTcBK, false, false);
+  QkSteps<0, D / 16>::run(tmem + half * 128, dq0 + (uint64_t)((half * TcSmem<D>::kTile) >> 4), dk, idq);
+  tc::commit(done);
+}
+
+// O_h (+)= P_h V: P_h from TMEM (aliasing S_h), V tile at descriptor dv; commits to `done`.
+template <int D>
+DMA_DEVINL void issue_pv(uint32_t tmem, int half, uint64_t dv, bool first, uint64_t* done) {
+  constexpr uint32_t idv = tc::idesc_bf16(128, D, false, true);
+  PvSteps<0, kTcBK / 16>::run(tmem + 256 + half * 128, tmem + half * 128, dv, idv, first ? 0u : 1u);
+  tc::commit(done);
+}
+
+// Item q of the heaviest-first order: pair kp (late pairs have the longest lists), row bh.
+struct Item { int bh, kp; };
+DMA_DEVINL Item item_of(int q, int BH, int n_pairs) { return Item{q % BH, n_pairs - 1 - q / BH}; }
+// The r-th item of CTA c among G: snake order over the CTAs, so that the CTAs that took the heavier
+// items of one round take the lighter ones of the next.
+DMA_DEVINL int item_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+
 template <int D, typename OutT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ counts, const int32_t* __restrict__ lists,
-                   const int32_t* __restrict__ list_je, const float* __restrict__ list_dl,
-                   OutT* __restrict__ O, float* __restrict__ LSE,
-                   int32_t* __restrict__ status, int H, int G, int N, int n_blocks, int list_cap,
+                   const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ pcounts,
+                   const int32_t* __restrict__ plists, const int32_t* __restrict__ pje,
+                   const float* __restrict__ pdl, OutT* __restrict__ O, float* __restrict__ LSE,
+                   int32_t* __restrict__ status, int BH, int H, int G, int N, int n_pairs, int pair_cap,
                    float scale_log2) {
   using S = TcSmem<D>;
   extern __shared__ __align__(1024) unsigned char sm[];
   TcBars& bar = *reinterpret_cast<TcBars*>(sm + S::kBars);
-  float* m_dl = reinterpret_cast<float*>(sm + S::kMeta);                        // [kMStages][128]
-  int32_t* m_je = reinterpret_cast<int32_t*>(sm + S::kMeta) + kMStages * kTcBK;  // [kMStages][128]
-  float* merge = reinterpret_cast<float*>(sm + S::kMerge);                       // [2][2][128]
-
-  const int kb = n_blocks - 1 - (int)blockIdx.x;   // heavy (late) blocks first
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh % H, g = h / G, Hkv = H / G;
-  const int t0 = kb * kBlockQ;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int32_t* cnt = counts + ((size_t)bh * n_blocks + kb) * 2;
-  const int n_full = cnt[0], n_live = cnt[1];
-  const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+  const int n_items = BH * n_pairs;
+  const int cta = blockIdx.x, n_ctas = gridDim.x;
   volatile int* abort_flag = &bar.abort_flag;
 
   if (tid == 0) {
@@ -145,20 +271,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       bar.abort_flag = 1;
     }
     tc::mbar_init(&bar.q_full, 32);
+    tc::mbar_init(&bar.q_empty, 1);
     for (int i = 0; i < kKStages; ++i) { tc::mbar_init(&bar.k_full[i], 32); tc::mbar_init(&bar.k_empty[i], 1); }
     for (int i = 0; i < kVStages; ++i) { tc::mbar_init(&bar.v_full[i], 32); tc::mbar_init(&bar.v_empty[i], 1); }
-    for (int i = 0; i < kMStages; ++i) {
-      tc::mbar_init(&bar.m_full[i], kProdThreads);
-      tc::mbar_init(&bar.m_empty[i], 128);
-    }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&bar.s_full[i], 1);
       tc::mbar_init(&bar.p_full[i], 128);
       tc::mbar_init(&bar.pv_done[i], 1);
     }
+    tc::mbar_init(&bar.drain, 1);
     tc::fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(&bar.tmem_base, 512);
     tc::tmem_relinquish();
   }
@@ -166,308 +290,349 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   __syncthreads();
   tc::fence_after();
   const uint32_t tmem = bar.tmem_base;
-  const bool run = n_tiles > 0 && !*abort_flag;
-  if (warp >= 8) {
-    regs_dec<kRegsOther>();   // warpgroups 2 and 3 give registers back
-  if (warp >= kProdWarp0) {
-    // ------------------------------------------------------------ producers (TMA gather4)
-    const int pw = warp - kProdWarp0;            // producer warp 0..3
-    const int prow = pw * 32 + lane;             // the tile row this thread owns
-    const int kvrow0 = (b * Hkv + g) * N;
-    const size_t lbase = ((size_t)bh * n_blocks + kb) * list_cap;
-    const int32_t* list = lists + lbase;
-    const int32_t* lje = list_je + lbase;
-    const float* ldl = list_dl + lbase;
-    constexpr uint32_t kRowBytes = D * 2;
-    const bool issuer = lane < 8;                // lanes 0-7 gather rows pw*32 + 4*lane .. +3
-    const uint32_t goff = (uint32_t)(pw * 32 + 4 * (lane & 7)) * 128;
-    if (run && issuer) {   // Q rows (rows past N repeat row N-1; their outputs are dropped)
-      int r[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) r[u] = bh * N + min(t0 + pw * 32 + 4 * lane + u, N - 1);
-      mbar_arrive_expect_tx(&bar.q_full, 4 * kRowBytes);
-#pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf)
-        tma_gather4(smem_u32(sm + S::kQ) + hf * 16384 + goff, &qmap, hf * 64, r[0], r[1], r[2], r[3], &bar.q_full);
-    }
-    // Software pipeline over tiles: this row's list entry and its metadata (written beside the list
-    // by the list kernel, so no load depends on another) are loaded two tiles ahead.
-    struct Entry { int j, je; float dl; };
-    auto entry_at = [&](int i) {
-      const int li = i * kTcBK + prow;
-      Entry x{-1, 0xffff, 0.f};
-      if (i < n_tiles && li < n_live) { x.j = list[li]; x.je = lje[li]; x.dl = ldl[li]; }
-      return x;
-    };
-    Entry ec = entry_at(0), en = entry_at(1);
-    int jv = -1;
-    for (int i = 0; run && i <= n_tiles; ++i) {
-      const Entry enn = entry_at(i + 2);
-      const int jc = ec.j;
-      if (i < n_tiles) {
-        const int ks = i % kKStages, ms = i % kMStages;
-        if (i >= kMStages &&
-            !wait_all(&bar.m_empty[ms], ((i / kMStages) - 1) & 1, abort_flag, status, kErrTimeoutMEmpty))
-          break;
-        m_dl[ms * kTcBK + prow] = ec.dl;
-        m_je[ms * kTcBK + prow] = ec.je;
-        tc::mbar_arrive(&bar.m_full[ms]);
-        if (i >= kKStages &&
-            !wait_all(&bar.k_empty[ks], ((i / kKStages) - 1) & 1, abort_flag, status, kErrTimeoutKEmpty))
-          break;
-        int r[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = __shfl_sync(0xffffffffu, jc, 4 * (lane & 7) + u);
-          r[u] = kvrow0 + (j >= 0 ? j : 0);
-        }
-        if (issuer) {
-          mbar_arrive_expect_tx(&bar.k_full[ks], 4 * kRowBytes);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf)
-            tma_gather4(smem_u32(sm + S::kK + ks * S::kTile) + hf * 16384 + goff, &kmap, hf * 64, r[0], r[1], r[2],
-                        r[3], &bar.k_full[ks]);
-        }
+  constexpr uint32_t kRowBytes = D * 2;
+
+  if (warp >= kMmaWarp) {
+    regs_dec<kRegsOther>();
+    if (warp >= kVWarp0) {
+      // ---------------------------------------------------------- producers (TMA gather4)
+      const bool kside = warp >= kKWarp0;
+      // row group (4 rows of a 128-row tile) of this lane, and whether the lane issues
+      int grp, ngrp;
+      if (kside) {
+        grp = (warp - kKWarp0) * 8 + lane;
+        ngrp = 8;
+      } else {
+        const int vw = warp - kVWarp0;
+        grp = vw * 11 + lane;
+        ngrp = vw < 2 ? 11 : 10;
       }
-      if (i >= 1) {
-        // V of tile i-1 (its stage belongs to the tile's stream)
-        const int vi = i - 1, vs = vi % kVStages;
-        if (vi >= kVStages &&
-            !wait_all(&bar.v_empty[vs], ((vi / kVStages) - 1) & 1, abort_flag, status, kErrTimeoutVEmpty))
-          break;
-        int r[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = __shfl_sync(0xffffffffu, jv, 4 * (lane & 7) + u);
-          r[u] = kvrow0 + (j >= 0 ? j : 0);
-        }
-        if (issuer) {
-          mbar_arrive_expect_tx(&bar.v_full[vs], 4 * kRowBytes);
-#pragma unroll
-          for (int hf = 0; hf < D / 64; ++hf)
-            tma_gather4(smem_u32(sm + S::kV + vs * S::kTile) + hf * 16384 + goff, &vmap, hf * 64, r[0], r[1], r[2],
-                        r[3], &bar.v_full[vs]);
-        }
-      }
-      jv = jc;
-      ec = en;
-      en = enn;
-    }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && run) {
-      constexpr uint32_t idq = tc::idesc_bf16(128, kTcBK, false, false);
-      constexpr uint32_t idv = tc::idesc_bf16(128, D, false, true);
-      const uint32_t qs = smem_u32(sm + S::kQ);
-      bool ok = tc::mbar_wait(&bar.q_full, 0, abort_flag, status, kErrTimeoutQ);
-      for (int i = 0; ok && i <= n_tiles; ++i) {
-        if (i < n_tiles) {   // S_x = Q K_i^T
-          const int x = i & 1, ks = i % kKStages;
-          if (!tc::mbar_wait(&bar.k_full[ks], (i / kKStages) & 1, abort_flag, status, kErrTimeoutK)) break;
-          if (i >= 2 && !tc::mbar_wait(&bar.pv_done[x], ((i >> 1) - 1) & 1, abort_flag, status, kErrTimeoutPV))
+      const bool issuer = lane < ngrp;
+      const uint32_t goff = (uint32_t)(4 * grp) * 128;
+      uint64_t* full = kside ? bar.k_full : bar.v_full;
+      uint64_t* empty = kside ? bar.k_empty : bar.v_empty;
+      const CUtensorMap* map = kside ? &kmap : &vmap;
+      const int tile_base = kside ? S::kK : S::kV;
+      const int err_empty = kside ? kErrTimeoutKEmpty : kErrTimeoutVEmpty;
+      int tc_count = 0;            // tiles issued by this role so far (stage = count % 2)
+      int n_done = 0;              // items done (Q buffer phase)
+      bool ok = !*abort_flag;
+      for (int r = 0; ok; ++r) {
+        const int q = item_index(r, cta, n_ctas);
+        if (q >= n_items) break;
+        const Item it = item_of(q, BH, n_pairs);
+        const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap;
+        const int n_live = pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1];
+        const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+        const int t0 = it.kp * 256;
+        const int b = it.bh / H, h = it.bh % H, g = h / G, Hkv = H / G;
+        const int kvrow0 = (b * Hkv + g) * N;
+        if (n_tiles == 0) continue;   // cannot happen: every query row selects at least one key
+        const int32_t* list = plists + lbase + 4 * grp;
+        int4 jn = make_int4(0, 0, 0, 0);
+        if (issuer) jn = *reinterpret_cast<const int4*>(list);
+        if (kside) {
+          // Q rows of both halves (rows past N repeat row N-1; their outputs are dropped)
+          if (n_done > 0 && !wait_all(&bar.q_empty, (n_done - 1) & 1, abort_flag, status, kErrTimeoutQEmpty)) {
+            ok = false;
             break;
-          tc::fence_after();
-          const uint32_t kbase = smem_u32(sm + S::kK + ks * S::kTile);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            tc::mma_bf16_ss(tmem + x * 128, tc::sdesc(qs + off, 16, 1024), tc::sdesc(kbase + off, 16, 1024), idq,
-                            kk > 0 ? 1u : 0u);
           }
-          tc::commit(&bar.s_full[x]);
-          tc::commit(&bar.k_empty[ks]);
-        }
-        if (i >= 1) {        // O_x += P_x V_{i-1}
-          const int pi = i - 1, x = pi & 1, vs = pi % kVStages;
-          if (!tc::mbar_wait(&bar.p_full[x], (pi >> 1) & 1, abort_flag, status, kErrTimeoutP)) break;
-          if (!tc::mbar_wait(&bar.v_full[vs], (pi / kVStages) & 1, abort_flag, status, kErrTimeoutV)) break;
-          tc::fence_after();
-          const uint32_t vbase = smem_u32(sm + S::kV + vs * S::kTile);
+          if (issuer) {
+            mbar_arrive_expect_tx(&bar.q_full, 8 * kRowBytes);
 #pragma unroll
-          for (int kk = 0; kk < kTcBK / 16; ++kk)
-            mma_bf16_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, tc::sdesc(vbase + kk * 2048, 16384, 1024),
-                        idv, (pi >= 2 || kk > 0) ? 1u : 0u);
-          tc::commit(&bar.pv_done[x]);
-          tc::commit(&bar.v_empty[vs]);
+            for (int qh = 0; qh < 2; ++qh) {
+              int rr[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) rr[u] = it.bh * N + min(t0 + qh * 128 + 4 * grp + u, N - 1);
+#pragma unroll
+              for (int hf = 0; hf < D / 64; ++hf)
+                tma_gather4(smem_u32(sm + S::kQ + qh * S::kTile) + hf * 16384 + goff, &qmap, hf * 64, rr[0], rr[1],
+                            rr[2], rr[3], &bar.q_full);
+            }
+          }
         }
+        for (int i = 0; i < n_tiles; ++i, ++tc_count) {
+          const int4 jc = jn;
+          if (issuer && i + 1 < n_tiles) jn = *reinterpret_cast<const int4*>(list + (i + 1) * kTcBK);
+          const int st = tc_count % 2;
+          if (tc_count >= 2 && !wait_all(&empty[st], ((tc_count / 2) - 1) & 1, abort_flag, status, err_empty)) {
+            ok = false;
+            break;
+          }
+          if (issuer) {
+            // padding entries (-1) fetch row 0 of the head: they are masked for every query row
+            const int r0 = kvrow0 + max(jc.x, 0), r1 = kvrow0 + max(jc.y, 0);
+            const int r2 = kvrow0 + max(jc.z, 0), r3 = kvrow0 + max(jc.w, 0);
+            mbar_arrive_expect_tx(&full[st], 4 * kRowBytes);
+#pragma unroll
+            for (int hf = 0; hf < D / 64; ++hf)
+              tma_gather4(smem_u32(sm + tile_base + st * S::kTile) + hf * 16384 + goff, map, hf * 64, r0, r1, r2, r3,
+                          &full[st]);
+          }
+        }
+        ++n_done;
       }
+      // after an abort: let this lane's copies in flight land before the CTA exits
+      if (!ok && issuer && tc_count > 0) drain_wait(&full[(tc_count - 1) % 2], ((tc_count - 1) / 2) & 1);
+    } else {
+      // ---------------------------------------------------------- MMA issuer (warp 8)
+      if (lane == 0) {
+        // descriptors of the operand bases
+        const uint64_t dq0 = tc::sdesc(smem_u32(sm + S::kQ), 16, 1024);
+        const uint64_t dk0 = tc::sdesc(smem_u32(sm + S::kK), 16, 1024);
+        const uint64_t dv0 = tc::sdesc(smem_u32(sm + S::kV), 16384, 1024);
+        int kc = 0, vc = 0;        // K / V tiles consumed
+        int tcount = 0;            // tiles done per half (S, P and PV completions of each half)
+        int n_done = 0;            // items done
+        bool ok = !*abort_flag;
+        for (int r = 0; ok; ++r) {
+          const int q = item_index(r, cta, n_ctas);
+          if (q >= n_items) break;
+          const Item it = item_of(q, BH, n_pairs);
+          const int n_live = pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1];
+          const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+          if (n_tiles == 0) continue;
+          if (!(ok = tc::mbar_wait(&bar.q_full, n_done & 1, abort_flag, status, kErrTimeoutQ))) break;
+          // first K tile: both halves
+          if (!(ok = tc::mbar_wait(&bar.k_full[kc % 2], (kc / 2) & 1, abort_flag, status, kErrTimeoutK))) break;
+          tc::fence_after();
+          for (int half = 0; half < 2 && ok; ++half) {
+            // S_h / P_h of the previous item is free once its last PV has completed
+            if (tcount > 0)
+              ok = tc::mbar_wait(&bar.pv_done[half], (tcount - 1) & 1, abort_flag, status, kErrTimeoutPV);
+            if (ok) issue_qk<D>(tmem, half, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[half]);
+          }
+          if (!ok) break;
+          tc::commit(&bar.k_empty[kc % 2]);
+          ++kc;
+          if (n_tiles == 1) tc::commit(&bar.q_empty);
+          for (int i = 0; i < n_tiles && ok; ++i) {
+            const int t = tcount + i;
+            const int vs = vc % 2;
+            ok = tc::mbar_wait(&bar.v_full[vs], (vc / 2) & 1, abort_flag, status, kErrTimeoutV) &&
+                 tc::mbar_wait(&bar.p_full[0], t & 1, abort_flag, status, kErrTimeoutP);
+            if (!ok) break;
+            tc::fence_after();
+            issue_pv<D>(tmem, 0, dv0 + (uint64_t)((vs * S::kTile) >> 4), i == 0, &bar.pv_done[0]);
+            const bool more = i + 1 < n_tiles;
+            if (more) {
+              ok = tc::mbar_wait(&bar.k_full[kc % 2], (kc / 2) & 1, abort_flag, status, kErrTimeoutK) &&
+                   tc::mbar_wait(&bar.pv_done[0], t & 1, abort_flag, status, kErrTimeoutPV);
+              if (!ok) break;
+              tc::fence_after();
+              issue_qk<D>(tmem, 0, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[0]);
+            }
+            if (!(ok = tc::mbar_wait(&bar.p_full[1], t & 1, abort_flag, status, kErrTimeoutP))) break;
+            tc::fence_after();
+            issue_pv<D>(tmem, 1, dv0 + (uint64_t)((vs * S::kTile) >> 4), i == 0, &bar.pv_done[1]);
+            tc::commit(&bar.v_empty[vs]);
+            ++vc;
+            if (more) {
+              if (!(ok = tc::mbar_wait(&bar.pv_done[1], t & 1, abort_flag, status, kErrTimeoutPV))) break;
+              tc::fence_after();
+              issue_qk<D>(tmem, 1, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[1]);
+              tc::commit(&bar.k_empty[kc % 2]);
+              ++kc;
+              if (i + 2 == n_tiles) tc::commit(&bar.q_empty);
+            }
+          }
+          tcount += n_tiles;
+          ++n_done;
+        }
+        // let every MMA issued so far complete before TMEM is released
+        tc::commit(&bar.drain);
+        drain_wait(&bar.drain, 0);
+      }
+      __syncwarp();
     }
-    __syncwarp();
-  }
   } else {
-    // ------------------------------------------------------------ softmax, stream x = warp / 4
+    // ------------------------------------------------------------ softmax, query half h = warp / 4
     regs_inc<kRegsSoftmax>();
-    const int x = warp >> 2;
+    const int h = warp >> 2;
     const int r = tid & 127;
-    const int t = t0 + r;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + x * 128 + lane_base, tO = tmem + 256 + x * 128 + lane_base;
-    float m_used = -INFINITY, l = 0.f;
-    int my_tiles = 0;
-    bool ok = run;
-    for (int i = x; ok && i < n_tiles; i += 2) {
-      const int k = i >> 1, ms = i % kMStages;
-      if (!wait_all(&bar.s_full[x], k & 1, abort_flag, status, kErrTimeoutS)) { ok = false; break; }
-      tc::fence_after();
-      uint32_t sr[kTcBK / 32][32];
+    const uint32_t tS = tmem + h * 128 + lane_base, tO = tmem + 256 + h * 128 + lane_base;
+    float* meta = reinterpret_cast<float*>(sm + S::kMeta) + h * 2 * 2 * kTcBK;   // [2 buffers][dl | je][128]
+    const uint64_t sc2 = f2(scale_log2, scale_log2);
+    int tcount = 0;
+    bool ok = !*abort_flag;
+    for (int rr = 0; ok; ++rr) {
+      const int q = item_index(rr, cta, n_ctas);
+      if (q >= n_items) break;
+      const Item it = item_of(q, BH, n_pairs);
+      const int32_t* cnt = pcounts + ((size_t)it.bh * n_pairs + it.kp) * 2;
+      const int n_full = cnt[0], n_live = cnt[1];
+      const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+      if (n_tiles == 0) continue;
+      const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap;
+      const int t = it.kp * 256 + h * 128 + r;   // this thread's query row
+      float dl_n = pdl[lbase + r];
+      int je_n = pje[lbase + r];
+      float m_used = -INFINITY, l = 0.f;
+      for (int i = 0; i < n_tiles; ++i) {
+        const int tt = tcount + i;
+        if (!wait_all(&bar.s_full[h], tt & 1, abort_flag, status, kErrTimeoutS)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after();
+        uint32_t sr[kTcBK / 32][32];
 #pragma unroll
-      for (int c = 0; c < kTcBK / 32; ++c) tc::tmem_ld32(tS + c * 32, sr[c]);
-      if (!wait_all(&bar.m_full[ms], (i / kMStages) & 1, abort_flag, status, kErrTimeoutM)) {
+        for (int c = 0; c < kTcBK / 32; ++c) tc::tmem_ld32(tS + c * 32, sr[c]);
+        // this tile's metadata: entry r from this thread, the others through the shared buffer
+        float* buf = meta + (i & 1) * 2 * kTcBK;
+        buf[r] = dl_n;
+        reinterpret_cast<int32_t*>(buf)[kTcBK + r] = je_n;
+        if (i + 1 < n_tiles) {
+          dl_n = pdl[lbase + (i + 1) * kTcBK + r];
+          je_n = pje[lbase + (i + 1) * kTcBK + r];
+        }
+        group_sync(h);
         tc::tmem_wait_ld();
+        const float4* dl4 = reinterpret_cast<const float4*>(buf);
+        const bool full_tile = (i + 1) * kTcBK <= n_full;
+        float mt = -INFINITY;
+        if (full_tile) {
+#pragma unroll
+          for (int c4 = 0; c4 < kTcBK / 4; ++c4) {
+            const float4 d = dl4[c4];
+            const int c = 4 * c4;
+            uint32_t* s4 = &sr[c / 32][c % 32];
+            const uint64_t va = f2_fma(f2(__uint_as_float(s4[0]), __uint_as_float(s4[1])), sc2, f2(d.x, d.y));
+            const uint64_t vb = f2_fma(f2(__uint_as_float(s4[2]), __uint_as_float(s4[3])), sc2, f2(d.z, d.w));
+            float v0, v1, v2, v3;
+            f2_split(va, v0, v1);
+            f2_split(vb, v2, v3);
+            mt = max3(mt, v0, v1);
+            mt = max3(mt, v2, v3);
+            s4[0] = __float_as_uint(v0);
+            s4[1] = __float_as_uint(v1);
+            s4[2] = __float_as_uint(v2);
+            s4[3] = __float_as_uint(v3);
+          }
+        } else {
+          const int4* je4 = reinterpret_cast<const int4*>(buf + kTcBK);
+#pragma unroll
+          for (int c4 = 0; c4 < kTcBK / 4; ++c4) {
+            const float4 d = dl4[c4];
+            const int4 w = je4[c4];
+            const int c = 4 * c4;
+            uint32_t* s4 = &sr[c / 32][c % 32];
+            const uint64_t va = f2_fma(f2(__uint_as_float(s4[0]), __uint_as_float(s4[1])), sc2, f2(d.x, d.y));
+            const uint64_t vb = f2_fma(f2(__uint_as_float(s4[2]), __uint_as_float(s4[3])), sc2, f2(d.z, d.w));
+            float v[4];
+            f2_split(va, v[0], v[1]);
+            f2_split(vb, v[2], v[3]);
+            const int ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int jj = (ww[u] << 16) >> 16, ee = ww[u] >> 16;   // key (-1: padding), e_j
+              v[u] = (jj <= t && t < ee) ? v[u] : -INFINITY;
+              s4[u] = __float_as_uint(v[u]);
+            }
+            mt = max3(mt, v[0], v[1]);
+            mt = max3(mt, v[2], v[3]);
+          }
+        }
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
+          alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
+          m_used = mt;
+          rescale = true;
+        }
+        const float base = m_used == -INFINITY ? 0.f : m_used;
+        const uint64_t nb2 = f2(-base, -base);
+        uint64_t psa = f2(0.f, 0.f), psb = f2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kTcBK / 64; ++c) {   // P (bf16 pairs) over columns [0, 64) of S_h
+          uint32_t pk[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int k0 = c * 64 + 2 * u;
+            const uint64_t x2 =
+                f2_add(f2(__uint_as_float(sr[k0 / 32][k0 % 32]), __uint_as_float(sr[k0 / 32][k0 % 32 + 1])), nb2);
+            float x0, x1, p0, p1;
+            f2_split(x2, x0, x1);
+            if (u % kPolyEvery == kPolyEvery - 1) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
+            if (u & 1) psb = f2_add(psb, f2(p0, p1));
+            else psa = f2_add(psa, f2(p0, p1));
+            pk[u] = pack_bf16x2(p0, p1);
+          }
+          tc::tmem_st32(tS + c * 32, pk);
+        }
+        // Rescale O_h now that the S row no longer occupies registers (PV of this tile waits for
+        // p_full).  O_h holds this item's tiles < i: their PV completed before S_h of tile i was
+        // computed.  The whole warp rescales when any of its rows needs it (alpha = 1 for the others).
+        if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orow[32];
+            tc::tmem_ld32(tO + c * 32, orow);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) orow[u] = __float_as_uint(__uint_as_float(orow[u]) * alpha);
+            tc::tmem_st32(tO + c * 32, orow);
+          }
+        }
+        float s0, s1, s2, s3;
+        f2_split(psa, s0, s1);
+        f2_split(psb, s2, s3);
+        l = l * alpha + ((s0 + s1) + (s2 + s3));
+        tc::tmem_wait_st();
+        tc::fence_before();
+        tc::mbar_arrive(&bar.p_full[h]);
+      }
+      if (!ok) break;
+      // ---- epilogue: O row = O_h / l, LSE = (m + log2 l) ln 2
+      const int last = tcount + n_tiles - 1;
+      if (!wait_all(&bar.pv_done[h], last & 1, abort_flag, status, kErrTimeoutPV)) {
         ok = false;
         break;
       }
-      tc::tmem_wait_ld();
-      const float4* dl4 = reinterpret_cast<const float4*>(m_dl + ms * kTcBK);
-      const bool full_tile = (i + 1) * kTcBK <= n_full;
-      float mt = -INFINITY;
-      if (full_tile) {
-#pragma unroll
-        for (int c4 = 0; c4 < kTcBK / 4; ++c4) {
-          const float4 d4 = dl4[c4];
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = c4 * 4 + u;
-            const float v = fmaf(__uint_as_float(sr[c / 32][c % 32]), scale_log2, dd[u]);
-            sr[c / 32][c % 32] = __float_as_uint(v);
-            mt = fmaxf(mt, v);
-          }
-        }
-      } else {
-        const int4* je4 = reinterpret_cast<const int4*>(m_je + ms * kTcBK);
-#pragma unroll
-        for (int c4 = 0; c4 < kTcBK / 4; ++c4) {
-          const float4 d4 = dl4[c4];
-          const int4 w4 = je4[c4];
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-          const int ww[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = c4 * 4 + u;
-            const int jj = (int)(int16_t)(ww[u] & 0xffff), ee = ww[u] >> 16;
-            float v = fmaf(__uint_as_float(sr[c / 32][c % 32]), scale_log2, dd[u]);
-            v = (jj >= 0 && jj <= t && t < ee) ? v : -INFINITY;
-            sr[c / 32][c % 32] = __float_as_uint(v);
-            mt = fmaxf(mt, v);
-          }
-        }
-      }
-      tc::mbar_arrive(&bar.m_empty[ms]);
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
-        alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
-        m_used = mt;
-        rescale = true;
-      }
-      // O_x is stable here: S_x of this tile was computed after the stream's previous PV finished.
-      // The whole warp rescales when any of its rows needs it (alpha = 1 for the others).
-      if (my_tiles > 0 && __any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orow[32];
-          tc::tmem_ld32(tO + c * 32, orow);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 32; ++u) orow[u] = __float_as_uint(__uint_as_float(orow[u]) * alpha);
-          tc::tmem_st32(tO + c * 32, orow);
-        }
-      }
-      const float base = m_used == -INFINITY ? 0.f : m_used;
-      float ps = 0.f;
-#pragma unroll
-      for (int c = 0; c < kTcBK / 64; ++c) {   // P (bf16 pairs) over columns [0, 64) of S_x
-        uint32_t pk[32];
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int k0 = c * 64 + 2 * u;
-          const float p0 = fast_exp2(__uint_as_float(sr[k0 / 32][k0 % 32]) - base);
-          const float p1 = fast_exp2(__uint_as_float(sr[(k0 + 1) / 32][(k0 + 1) % 32]) - base);
-          ps += p0 + p1;
-          pk[u] = pack_bf16x2(p0, p1);
-        }
-        tc::tmem_st32(tS + c * 32, pk);
-      }
-      l = l * alpha + ps;
-      tc::tmem_wait_st();
-      tc::fence_before();
-      tc::mbar_arrive(&bar.p_full[x]);
-      ++my_tiles;
-    }
-    // ---- merge the two streams
-    // wait for this stream's last PV
-    bool done = ok;
-    if (ok && my_tiles > 0) {
-      const int last = x + 2 * (my_tiles - 1);
-      done = wait_all(&bar.pv_done[x], (last >> 1) & 1, abort_flag, status, kErrTimeoutPV);
-    }
-    merge[(x * 2 + 0) * 128 + r] = m_used;
-    merge[(x * 2 + 1) * 128 + r] = l;
-    softmax_sync();
-    const float m0 = merge[0 * 128 + r], l0 = merge[1 * 128 + r];
-    const float m1 = merge[2 * 128 + r], l1 = merge[3 * 128 + r];
-    const float M = fmaxf(m0, m1);
-    const float Mb = M == -INFINITY ? 0.f : M;
-    const float s0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - Mb), s1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - Mb);
-    const float L = l0 * s0 + l1 * s1;
-    const bool have1 = n_tiles > 1;   // stream B has at least one tile
-    // stream B scales its O rows in place; stream A then writes (O_A s0 + O_B') / L
-    if (x == 1 && have1 && __all_sync(0xffffffffu, done)) {
       tc::fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const bool valid = t < N;
+      OutT* orow = O + ((size_t)it.bh * N + (valid ? t : 0)) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
         tc::tmem_ld32(tO + c * 32, ov);
         tc::tmem_wait_ld();
-#pragma unroll
-        for (int u = 0; u < 32; ++u) ov[u] = __float_as_uint(__uint_as_float(ov[u]) * s1);
-        tc::tmem_st32(tO + c * 32, ov);
-      }
-      tc::tmem_wait_st();
-    }
-    tc::fence_before();
-    softmax_sync();
-    tc::fence_after();
-    if (x == 0 && run && __all_sync(0xffffffffu, done && !*abort_flag)) {
-      const uint32_t tO1 = tmem + 384 + lane_base;
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      OutT* orow = O + ((size_t)bh * N + t) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t oa[32], ob[32];
-        tc::tmem_ld32(tO + c * 32, oa);
-        if (have1) tc::tmem_ld32(tO1 + c * 32, ob);
-        tc::tmem_wait_ld();
-        float of[32];
-#pragma unroll
-        for (int u = 0; u < 32; ++u)
-          of[u] = (__uint_as_float(oa[u]) * s0 + (have1 ? __uint_as_float(ob[u]) : 0.f)) * inv;
-        if (t < N) {
+        if (valid) {
           if constexpr (sizeof(OutT) == 2) {
 #pragma unroll
             for (int u = 0; u < 32; u += 8) {
               uint4 v;
-              v.x = pack_bf16x2(of[u], of[u + 1]);
-              v.y = pack_bf16x2(of[u + 2], of[u + 3]);
-              v.z = pack_bf16x2(of[u + 4], of[u + 5]);
-              v.w = pack_bf16x2(of[u + 6], of[u + 7]);
+              v.x = pack_bf16x2(__uint_as_float(ov[u]) * inv, __uint_as_float(ov[u + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(ov[u + 2]) * inv, __uint_as_float(ov[u + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(ov[u + 4]) * inv, __uint_as_float(ov[u + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(ov[u + 6]) * inv, __uint_as_float(ov[u + 7]) * inv);
               *reinterpret_cast<uint4*>(orow + c * 32 + u) = v;
             }
           } else {
 #pragma unroll
             for (int u = 0; u < 32; u += 4)
-              *reinterpret_cast<float4*>(orow + c * 32 + u) = make_float4(of[u], of[u + 1], of[u + 2], of[u + 3]);
+              *reinterpret_cast<float4*>(orow + c * 32 + u) =
+                  make_float4(__uint_as_float(ov[u]) * inv, __uint_as_float(ov[u + 1]) * inv,
+                              __uint_as_float(ov[u + 2]) * inv, __uint_as_float(ov[u + 3]) * inv);
           }
         }
       }
-      if (t < N) LSE[(size_t)bh * N + t] = (Mb + __log2f(L)) * kLn2;
+      if (valid) LSE[(size_t)it.bh * N + t] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
+      tc::fence_before();
+      tcount += n_tiles;
     }
   }
   tc::fence_before();
   __syncthreads();
   tc::fence_after();
-  if (warp == 8) tc::tmem_dealloc(tmem, 512);
+  if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- host side: tensor maps
@@ -483,6 +648,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   return fn;
+}
+
+// SMs of the current device (cached per device).
+int sm_count() {
+  static std::mutex mu;
+  static int count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    count[dev] = n;
+  }
+  return count[dev];
 }
 
 // 2-D view [rows, d] of a row-major bf16 tensor; boxes of 64 columns x 1 row (the gather4 form),
@@ -510,15 +690,16 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
   auto k = attn_fwd_tc_kernel<D, OutT>;
   const int smem = TcSmem<D>::kBytes;
   { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
-  dim3 grid(P.n_blocks, P.B * P.H);
+  // persistent: one CTA per SM (the shared-memory footprint admits one), at most one per item
+  const int n_items = P.B * P.H * P.n_pairs;
+  const int grid = n_items < sm_count() ? n_items : sm_count();
   // delta and e enter through the per-entry metadata that the list kernel wrote beside the lists
   (void)delta;
   (void)evict;
-  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
-                                   ws_ptr<int32_t>(ws, P.off_list_je), ws_ptr<float>(ws, P.off_list_dl),
-                                   (OutT*)O, LSE,
-                                   ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_blocks, P.list_cap,
-                                   P.scale * kLog2e);
+  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists),
+                                   ws_ptr<int32_t>(ws, P.off_pje), ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE,
+                                   ws_ptr<int32_t>(ws, P.off_status), P.B * P.H, P.H, P.G, P.N, P.n_pairs,
+                                   P.pair_cap, P.scale * kLog2e);
   return cudaGetLastError();
 }
 

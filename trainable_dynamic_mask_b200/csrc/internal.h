@@ -10,6 +10,7 @@
 namespace dma {
 
 constexpr int kBlockQ = DMA_BLOCK_Q;   // query rows per block of the mask encoding
+constexpr int kPairQ = 2 * kBlockQ;    // query rows per attention-forward work item
 constexpr int kTopwMaxN = 16384;      // prefill/training selection keeps a whole row in SMEM
 constexpr int kDecodeSplit = 256;      // selected keys per decode split
 constexpr int kGateSlice = 512;        // positions per partial sum of dDelta
@@ -24,6 +25,8 @@ struct Plan {
   bool decode;    // Nq == 1 and N > 1 ... the single query sits at position N-1
   int n_blocks;   // query blocks of kBlockQ rows (prefill)
   int list_cap;   // entries per block list
+  int n_pairs;    // query blocks of kPairQ rows (attention forward work items)
+  int pair_cap;   // entries per pair list (a multiple of 128; every list is padded to 128)
   int sel_len;    // decode: min(w, N)
   int n_split;    // decode: splits per (b, h)
   int n_slices;   // gate backward: position slices of kGateSlice
@@ -34,7 +37,9 @@ struct Plan {
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
   size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
-  size_t off_list_je, off_list_dl;     // per list entry: j | e_j << 16 (i32), delta_j * log2(e) (f32)
+  // attention forward: live-key lists of query pairs of blocks (kPairQ rows), each entry with its
+  // j | e_j << 16 (i32) and delta_j * log2(e) (f32); [B, H, n_pairs, pair_cap], counts [.., 2]
+  size_t off_pcounts, off_plists, off_pje, off_pdl;
   size_t off_gx;                       // gate backward: gx [B, H, N] f32
   size_t off_dA_part;                  // gate backward: [B*H][ceil(N/1024)] f32
   size_t off_dDelta_part;              // gate backward: [n_slices*B][Hkv*d][H] f32

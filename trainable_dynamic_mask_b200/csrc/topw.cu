@@ -323,25 +323,48 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   }
 }
 
-// Live keys of query block k: j < t1 and e_j > max(j, t0).  Full keys (j <= t0, e_j >= t1) first.
+// Live keys of a range of query rows [t0, t1): j < t1 and e_j > max(j, t0).  The "full" ones
+// (j <= t0 and e_j >= t1: selected by every row of the range) come first, then the others, each
+// group in ascending key order.  One CTA scans the keys of a pair of blocks (kPairQ rows) once and
+// builds three lists from them: those of its two blocks (the mask encoding of the interface) and
+// that of the pair (the attention forward's work item), whose entries also carry j | e_j << 16
+// and delta_j * log2(e) and which is padded to a multiple of 128 entries with key -1 (masked for
+// every row: e = 0).
 constexpr int kListThreads = 256;
+constexpr int kListWarps = kListThreads / 32;
+constexpr int kListBits = 10;                    // packed per-warp counters (a warp counts <= 128)
+constexpr int kListMask = (1 << kListBits) - 1;
 
 __global__ void __launch_bounds__(kListThreads)
 topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
-                  int32_t* __restrict__ counts, int32_t* __restrict__ lists, int32_t* __restrict__ list_je,
-                  float* __restrict__ list_dl, int N, int list_cap, int n_blocks) {
-  __shared__ int32_t partial[2 * kC];
-  __shared__ int32_t wsum[2][kListThreads / 32];
-  const int k = blockIdx.x, row = blockIdx.y;
+                  int32_t* __restrict__ counts, int32_t* __restrict__ lists,
+                  int32_t* __restrict__ pcounts, int32_t* __restrict__ plists,
+                  int32_t* __restrict__ pje, float* __restrict__ pdl, int N, int list_cap, int pair_cap,
+                  int n_blocks, int n_pairs) {
+  // partial keys: block a (<= 2C), block b (<= 2C), pair (<= 4C)
+  __shared__ int32_t part[8 * kC];
+  __shared__ int32_t wsum[6][kListWarps];   // per warp: full count of list 0..2, partial count of 0..2
+  const int kp = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = k * kC, t1 = min(t0 + kC, N);
+  const int t0 = kp * kPairQ;
+  const bool has_b = t0 + kC < N;
+  // list 0: block 2kp, list 1: block 2kp + 1, list 2: the pair
+  const int lo[3] = {t0, t0 + kC, t0};
+  const int hi[3] = {min(t0 + kC, N), min(t0 + kPairQ, N), min(t0 + kPairQ, N)};
+  const int pcap[3] = {2 * kC, 2 * kC, 4 * kC};
+  const int poff[3] = {0, 2 * kC, 4 * kC};
+  const int cap[3] = {list_cap, list_cap, pair_cap};
+  const int t1 = hi[2];
   const int32_t* erow = evict + (size_t)row * N;
-  const size_t lbase = ((size_t)row * n_blocks + k) * list_cap;
-  int32_t* out = lists + lbase;
-  int32_t* oje = list_je + lbase;   // j | e_j << 16 of each entry (what the attention kernel tests)
-  float* odl = list_dl + lbase;     // delta_j * log2(e)
   const float* drow = delta + (size_t)row * N;
-  int nfull = 0, npart = 0;
+  int32_t* out[3];
+  out[0] = lists + ((size_t)row * n_blocks + 2 * kp) * list_cap;
+  out[1] = has_b ? out[0] + list_cap : out[0];
+  const size_t pbase = ((size_t)row * n_pairs + kp) * pair_cap;
+  out[2] = plists + pbase;
+  int32_t* oje = pje + pbase;
+  float* odl = pdl + pbase;
+  int nfull[3] = {0, 0, 0}, npart[3] = {0, 0, 0};
   int enext[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -349,78 +372,125 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
     enext[u] = j < t1 ? erow[j] : 0;
   }
   for (int base = 0; base < t1; base += kListThreads * 4) {
-    int f[4], q[4], ecur[4];
-    int cf = 0, cq = 0;
+    int ecur[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       ecur[u] = enext[u];
       const int jn = base + kListThreads * 4 + tid * 4 + u;   // prefetch the next round
       enext[u] = jn < t1 ? erow[jn] : 0;
     }
+    int cf = 0, cq = 0;              // packed counts of this thread's full / partial keys
+    uint32_t fbits = 0, qbits = 0;   // bit 3u + L: key u is full / partial in list L
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = base + tid * 4 + u;
       const int e = ecur[u];
-      const bool live = j < t1 && e > max(j, t0);
-      const bool full = live && j <= t0 && e >= t1;
-      f[u] = full;
-      q[u] = live && !full;
-      cf += f[u];
-      cq += q[u];
+#pragma unroll
+      for (int L = 0; L < 3; ++L) {
+        const bool valid = L != 1 || has_b;
+        const bool live = valid && j < hi[L] && e > max(j, lo[L]);
+        const bool full = live && j <= lo[L] && e >= hi[L];
+        fbits |= (uint32_t)full << (3 * u + L);
+        qbits |= (uint32_t)(live && !full) << (3 * u + L);
+        cf += (int)full << (kListBits * L);
+        cq += (int)(live && !full) << (kListBits * L);
+      }
     }
     int incf = cf, incq = cq;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      int yf = __shfl_up_sync(0xffffffffu, incf, o);
-      int yq = __shfl_up_sync(0xffffffffu, incq, o);
+      const int yf = __shfl_up_sync(0xffffffffu, incf, o);
+      const int yq = __shfl_up_sync(0xffffffffu, incq, o);
       if (lane >= o) { incf += yf; incq += yq; }
     }
-    if (lane == 31) { wsum[0][warp] = incf; wsum[1][warp] = incq; }
-    __syncthreads();
-    int wf = 0, wq = 0, tf = 0, tq = 0;
-    for (int i = 0; i < kListThreads / 32; ++i) {
-      if (i < warp) { wf += wsum[0][i]; wq += wsum[1][i]; }
-      tf += wsum[0][i];
-      tq += wsum[1][i];
+    if (lane == 31) {
+#pragma unroll
+      for (int L = 0; L < 3; ++L) {
+        wsum[L][warp] = (incf >> (kListBits * L)) & kListMask;
+        wsum[3 + L][warp] = (incq >> (kListBits * L)) & kListMask;
+      }
     }
-    int of = nfull + wf + incf - cf, oq = npart + wq + incq - cq;
+    __syncthreads();
+    int of[3], oq[3], tf[3], tq[3];
+#pragma unroll
+    for (int L = 0; L < 3; ++L) {
+      int bf = 0, bq = 0, sf = 0, sq = 0;
+      for (int i = 0; i < kListWarps; ++i) {
+        const int vf = wsum[L][i], vq = wsum[3 + L][i];
+        if (i < warp) { bf += vf; bq += vq; }
+        sf += vf;
+        sq += vq;
+      }
+      of[L] = nfull[L] + bf + (((incf - cf) >> (kListBits * L)) & kListMask);
+      oq[L] = npart[L] + bq + (((incq - cq) >> (kListBits * L)) & kListMask);
+      tf[L] = sf;
+      tq[L] = sq;
+    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = base + tid * 4 + u;
-      if (f[u]) {
-        if (of < list_cap) {
-          out[of] = j;
-          oje[of] = (j & 0xffff) | (ecur[u] << 16);
-          odl[of] = drow[j] * kLog2e;
+#pragma unroll
+      for (int L = 0; L < 3; ++L) {
+        if ((fbits >> (3 * u + L)) & 1u) {
+          if (of[L] < cap[L]) {
+            out[L][of[L]] = j;
+            if (L == 2) {
+              oje[of[L]] = (j & 0xffff) | (ecur[u] << 16);
+              odl[of[L]] = drow[j] * kLog2e;
+            }
+          }
+          ++of[L];
         }
-        ++of;
+        if ((qbits >> (3 * u + L)) & 1u) {
+          if (oq[L] < pcap[L]) part[poff[L] + oq[L]] = j;
+          ++oq[L];
+        }
       }
-      if (q[u]) { if (oq < 2 * kC) partial[oq] = j; ++oq; }
     }
-    nfull += tf;
-    npart += tq;
-    __syncthreads();
+#pragma unroll
+    for (int L = 0; L < 3; ++L) {
+      nfull[L] += tf[L];
+      npart[L] += tq[L];
+    }
+    __syncthreads();   // wsum is rewritten next round
   }
-  // at most C evicted old keys plus C new keys; a live set never exceeds list_cap
-  nfull = min(nfull, list_cap);
-  npart = min(min(npart, 2 * kC), list_cap - nfull);
-  for (int i = tid; i < npart; i += kListThreads) {
-    const int j = partial[i];
-    out[nfull + i] = j;
-    oje[nfull + i] = (j & 0xffff) | (erow[j] << 16);
-    odl[nfull + i] = drow[j] * kLog2e;
+  // Caps: a block list holds at most w live keys at its first row plus C new ones (<= list_cap);
+  // its partial keys are at most C evicted plus C new ones.  A pair: w + 2C and 2C + 2C.
+#pragma unroll
+  for (int L = 0; L < 3; ++L) {
+    nfull[L] = min(nfull[L], cap[L]);
+    npart[L] = min(min(npart[L], pcap[L]), cap[L] - nfull[L]);
   }
-  // pad the last 128-entry tile: key -1 is masked everywhere
-  const int nlive = nfull + npart;
-  const int nround = min(list_cap, (nlive + kC - 1) / kC * kC);
+#pragma unroll
+  for (int L = 0; L < 3; ++L) {
+    if (L == 1 && !has_b) continue;
+    for (int i = tid; i < npart[L]; i += kListThreads) {
+      const int j = part[poff[L] + i];
+      out[L][nfull[L] + i] = j;
+      if (L == 2) {
+        oje[nfull[L] + i] = (j & 0xffff) | (erow[j] << 16);
+        odl[nfull[L] + i] = drow[j] * kLog2e;
+      }
+    }
+  }
+  const int nlive = nfull[2] + npart[2];
+  const int nround = min(pair_cap, (nlive + kC - 1) / kC * kC);
   for (int i = nlive + tid; i < nround; i += kListThreads) {
-    out[i] = -1;
+    out[2][i] = -1;
     oje[i] = 0xffff;
     odl[i] = 0.f;
   }
   if (tid == 0) {
-    counts[((size_t)row * n_blocks + k) * 2 + 0] = nfull;
-    counts[((size_t)row * n_blocks + k) * 2 + 1] = nfull + npart;
+    int32_t* ca = counts + ((size_t)row * n_blocks + 2 * kp) * 2;
+    ca[0] = nfull[0];
+    ca[1] = nfull[0] + npart[0];
+    if (has_b) {
+      ca[2] = nfull[1];
+      ca[3] = nfull[1] + npart[1];
+    }
+    int32_t* cp = pcounts + ((size_t)row * n_pairs + kp) * 2;
+    cp[0] = nfull[2];
+    cp[1] = nlive;
   }
 }
 
@@ -541,9 +611,10 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   topw_sort_kernel<<<rows, kSortThreads2, smem, s>>>(delta, pbuf, rbuf, Tbuf, P.N, P.w);
   topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
-  topw_lists_kernel<<<dim3(P.n_blocks, rows), kListThreads, 0, s>>>(
+  topw_lists_kernel<<<dim3(P.n_pairs, rows), kListThreads, 0, s>>>(
       evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
-      ws_ptr<int32_t>(ws, P.off_list_je), ws_ptr<float>(ws, P.off_list_dl), P.N, P.list_cap, P.n_blocks);
+      ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_pje),
+      ws_ptr<float>(ws, P.off_pdl), P.N, P.list_cap, P.pair_cap, P.n_blocks, P.n_pairs);
   return cudaGetLastError();
 }
 
