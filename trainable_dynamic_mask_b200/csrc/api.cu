@@ -105,6 +105,10 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));
     R.off_tw_T = take(BH * (R.n_blocks + 1) * sizeof(int32_t));
+    {
+      const size_t L = (size_t)topw_seg_len(R.N);
+      R.off_tw_keys = take(BH * ((R.N + L - 1) / L) * L * sizeof(uint64_t));
+    }
   } else {
     R.off_sel = take(BH * R.sel_len * sizeof(int32_t));
     R.off_dec_part = take(BH * R.n_split * (size_t)(R.d + 2) * sizeof(float));

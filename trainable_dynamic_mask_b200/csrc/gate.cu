@@ -272,6 +272,118 @@ __global__ void gate_bwd_reduce_kernel(const float* __restrict__ part, const flo
   }
 }
 
+// bf16 values: x = v_cat Delta as a [positions x Hkv*d] x [Hkv*d x H] product on the tensor cores
+// (mma.sync m16n8k16, float32 accumulation; bf16 products are exact in float32).  CTA = 16 key
+// positions of one batch row, 8 warps splitting the reduction in 16-wide steps (step s to warp
+// s % 8); the 8 partial [16 x H] tiles are summed through shared memory.  The V rows of the 16
+// positions (all Hkv heads: 16 rows of Hkv*d) and Delta (zero-padded to HT*8 columns) are staged
+// with coalesced 16-byte loads; A fragments come from a 16-byte-chunk XOR swizzle (conflict-free
+// ldmatrix), B fragments from ldmatrix.trans of the row-major Delta.
+constexpr int kGmP = 16;
+constexpr int kGmThreads = 256;
+
+template <int HT>   // Delta column tiles of 8 (H <= 8 * HT), HT even
+__global__ void __launch_bounds__(kGmThreads)
+gate_fwd_mma_kernel(const uint16_t* __restrict__ V, const uint16_t* __restrict__ Delta, const float* __restrict__ A,
+                    float* __restrict__ delta, float* __restrict__ x_save, int H, int Hkv, int N, int d) {
+  extern __shared__ __align__(128) unsigned char gsm[];
+  const int K = Hkv * d, KC = K / 8;                        // reduction length, its 16-byte chunks
+  uint16_t* Vs = reinterpret_cast<uint16_t*>(gsm);          // [16][K], chunk c of row p at c ^ (p & 7)
+  uint16_t* Ds = Vs + kGmP * K;                             // [K][8 HT]
+  float* red = reinterpret_cast<float*>(Ds + (size_t)K * 8 * HT);   // [8 warps][16][8 HT]
+  const int b = blockIdx.y, p0 = blockIdx.x * kGmP;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int dch = d / 8;
+  // ---- stage V (16 positions x K) and Delta (K x H, padded to 8 HT columns)
+  for (int q = tid; q < kGmP * KC; q += kGmThreads) {
+    const int p = q / KC, kc = q % KC;
+    const int g = kc / dch, c = kc % dch;
+    const int pos = p0 + p;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (pos < N) v = *reinterpret_cast<const uint4*>(V + ((size_t)(b * Hkv + g) * N + pos) * d + c * 8);
+    *reinterpret_cast<uint4*>(Vs + (size_t)p * K + ((kc ^ (p & 7)) * 8)) = v;
+  }
+  if ((H & 7) == 0) {
+    const int hc = H / 8;
+    for (int q = tid; q < K * HT; q += kGmThreads) {
+      const int r = q / HT, c = q % HT;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (c < hc) v = *reinterpret_cast<const uint4*>(Delta + (size_t)r * H + c * 8);
+      *reinterpret_cast<uint4*>(Ds + (size_t)r * 8 * HT + c * 8) = v;
+    }
+  } else {
+    for (int q = tid; q < K * 8 * HT; q += kGmThreads) {
+      const int r = q / (8 * HT), h = q % (8 * HT);
+      Ds[q] = h < H ? Delta[(size_t)r * H + h] : (uint16_t)0;
+    }
+  }
+  __syncthreads();
+  // ---- partial products over this warp's reduction steps
+  float acc[HT][4];
+#pragma unroll
+  for (int n = 0; n < HT; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+  const uint32_t vs_base = smem_u32(Vs), ds_base = smem_u32(Ds);
+  const int arow = lane & 15, achunk = lane >> 4;               // ldmatrix.x4 address of this lane
+  const int brow = (lane & 7) + ((lane >> 3) & 1) * 8, btile = lane >> 4;
+  for (int ks = warp; ks < K / 16; ks += 8) {
+    uint32_t a[4];
+    const int kc = ks * 2 + achunk;
+    ldmatrix_x4(vs_base + (uint32_t)(arow * K + ((kc ^ (arow & 7)) * 8)) * 2, a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int n = 0; n < HT; n += 2) {
+      uint32_t b0, b1, b2, b3;
+      ldmatrix_x4_trans(ds_base + (uint32_t)((ks * 16 + brow) * 8 * HT + (n + btile) * 8) * 2, b0, b1, b2, b3);
+      mma_bf16_16816(acc[n], a, b0, b1);
+      mma_bf16_16816(acc[n + 1], a, b2, b3);
+    }
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < HT; ++n) {
+    float* rw = red + (size_t)warp * kGmP * 8 * HT;
+    rw[g * 8 * HT + n * 8 + 2 * t] = acc[n][0];
+    rw[g * 8 * HT + n * 8 + 2 * t + 1] = acc[n][1];
+    rw[(g + 8) * 8 * HT + n * 8 + 2 * t] = acc[n][2];
+    rw[(g + 8) * 8 * HT + n * 8 + 2 * t + 1] = acc[n][3];
+  }
+  __syncthreads();
+  for (int o = tid; o < kGmP * H; o += kGmThreads) {
+    const int p = o / H, h = o % H;
+    const int pos = p0 + p;
+    if (pos >= N) continue;
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) x += red[((size_t)w * kGmP + p) * 8 * HT + h];
+    const size_t off = (size_t)(b * H + h) * N + pos;
+    delta[off] = expf(A[h] * softplus_f(x));
+    if (x_save) x_save[off] = x;
+  }
+}
+
+template <int HT>
+cudaError_t launch_gate_fwd_mma(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
+                                float* x_save, cudaStream_t s) {
+  const int K = P.Hkv * P.d;
+  const size_t smem = (size_t)kGmP * K * 2 + (size_t)K * 8 * HT * 2 + (size_t)8 * kGmP * 8 * HT * 4;
+  auto k = gate_fwd_mma_kernel<HT>;
+  { cudaError_t ea = ensure_smem_limit(k, (int)smem); if (ea != cudaSuccess) return ea; }
+  dim3 grid((P.N + kGmP - 1) / kGmP, P.B);
+  k<<<grid, kGmThreads, smem, s>>>((const uint16_t*)V, (const uint16_t*)Delta, A, delta, x_save, P.H, P.Hkv, P.N,
+                                   P.d);
+  return cudaGetLastError();
+}
+
+// Shared memory of the tensor-core gate for problem P (0 when it does not apply).
+size_t gate_mma_smem(const Plan& P) {
+  if (!P.bf16 || P.H > 64) return 0;
+  const int HT = P.H <= 16 ? 2 : P.H <= 32 ? 4 : 8;
+  const size_t K = (size_t)P.Hkv * P.d;
+  const size_t smem = kGmP * K * 2 + K * 8 * HT * 2 + (size_t)8 * kGmP * 8 * HT * 4;
+  return smem <= 200 * 1024 ? smem : 0;
+}
+
 template <typename T, int HPT>
 cudaError_t launch_gate_fwd_t(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
                               float* x_save, cudaStream_t s) {
@@ -299,6 +411,11 @@ cudaError_t launch_gate_fwd_h(const Plan& P, const void* V, const void* Delta, c
 
 cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             float* delta, float* x_save, cudaStream_t s) {
+  if (gate_mma_smem(P) > 0) {
+    if (P.H <= 16) return launch_gate_fwd_mma<2>(P, V, Delta, A, delta, x_save, s);
+    if (P.H <= 32) return launch_gate_fwd_mma<4>(P, V, Delta, A, delta, x_save, s);
+    return launch_gate_fwd_mma<8>(P, V, Delta, A, delta, x_save, s);
+  }
   return P.bf16 ? launch_gate_fwd_h<uint16_t>(P, V, Delta, A, delta, x_save, s)
                 : launch_gate_fwd_h<float>(P, V, Delta, A, delta, x_save, s);
 }

@@ -17,6 +17,9 @@ constexpr int kGateSlice = 512;        // positions per partial sum of dDelta
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Segment length of the top-w rank computation for a row of N keys: about 8 segments per row.
+inline int topw_seg_len(int N) { return N <= 4096 ? 512 : N <= 8192 ? 1024 : 2048; }
+
 // Resolved problem and workspace plan.
 struct Plan {
   int B, H, Hkv, N, Nq, d, w, G;
@@ -37,6 +40,7 @@ struct Plan {
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
   size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
+  size_t off_tw_keys;                  // top-w: sorted segments of composite keys [B, H, npad] u64
   // attention forward: live-key lists of query pairs of blocks (kPairQ rows), each entry with its
   // j | e_j << 16 (i32) and delta_j * log2(e) (f32); [B, H, n_pairs, pair_cap], counts [.., 2]
   size_t off_pcounts, off_plists, off_pje, off_pdl;

@@ -9,9 +9,11 @@
 // with t: key j is selected exactly for t in [j, e_j).  The prefill kernels compute e for every key
 // and, per block of DMA_BLOCK_Q queries, the list of keys live in the block.
 //
-// Algorithm (one CTA per (b, h) row, the row resident in shared memory):
-//  1. stable LSD radix sort of the row by (delta desc, index asc): p[r] = position of rank r,
-//     rank[j] = rank of position j (rank 0 = best);
+// Algorithm:
+//  1. ranks of the row in the order (delta desc, index asc): the row's composite keys are cut into
+//     segments, each segment sorted by its own CTA, and a key's rank is the number of smaller keys
+//     over all sorted segments: p[r] = position of rank r, rank[j] = rank of position j (rank 0 =
+//     best);
 //  2. T_k = rank of the w-th best key among positions [0, kC) for every chunk boundary k
 //     (C = 128), from a [rank bucket][position chunk] count table with prefix sums over chunks
 //     (T_k = N when kC <= w: nothing evicted yet);
@@ -20,10 +22,10 @@
 //     e = max(j, first t >= kC at which #{i <= t : rank_i < r} reaches w), where the count of old
 //     keys better than r follows from T_k and the sorted candidate list.  New keys that survive to
 //     the end (rank <= T at the last boundary) get e = N.  Every key's e is written exactly once.
-// A second kernel (one CTA per (row, query block)) compacts the live keys of each block:
-// full keys (selected by every existing row: j <= t0 and e_j >= min(t0 + C, N)) first, then the
-// partial ones (at most 2C: keys evicted inside the block and the block's own keys), each in
-// ascending order.
+//  4. one CTA per (row, pair of query blocks) compacts the live keys of the two blocks and of the
+//     pair: full keys (selected by every existing row of the range: j <= t0 and e_j >= t1) first,
+//     then the partial ones (keys evicted inside the range and the range's own keys), each in
+//     ascending order.
 #include "common.cuh"
 
 namespace dma {
@@ -43,149 +45,106 @@ DMA_DEVINL int nth_set_bit(uint32_t x, int n) {
   return __ffs(x) - 1;
 }
 
-// ---------------------------------------------------------------- sort + thresholds (per row)
+// ---------------------------------------------------------------- ranks + thresholds (per row)
+//
+// The order (delta descending, index ascending) is that of the 64-bit composite key
+// (~order_key(delta_j)) << 32 | j taken ascending; the keys of a row are distinct.  A row is cut
+// into nseg segments of L keys (padding keys 2^64 - 1 sort last); each segment is sorted by one CTA
+// (bitonic network in shared memory), then the rank of a key is the number of smaller keys summed
+// over the sorted segments (its own index in its segment plus a lower bound in every other one).
+// Many CTAs per row keep the SMs busy even for a few (b, h) rows.
 
-constexpr int kSortThreads2 = 1024;
-constexpr int kSortWarps2 = kSortThreads2 / 32;
-constexpr int kMaxItems = kTopwMaxN / kSortThreads2;   // 16 keys per thread at most
+DMA_DEVINL uint64_t topw_key(float delta, int j) {
+  return ((uint64_t)(~order_key(delta)) << 32) | (uint32_t)j;
+}
 
-// Shared-memory index with one pad word every 32: thread t's run [IT*t, IT*t + IT) starts in a
-// different bank for every lane of a warp when IT is a power of two.
-DMA_DEVINL int pad32(int i) { return i + (i >> 5); }
-
-// One CTA per (b, h) row: stable LSD radix sort of the row by (delta descending, index ascending)
-// with 4-bit digits, thread-private digit counters and a block-wide scan per pass (digit positions
-// where every key agrees are skipped); then the threshold ranks T_k for every chunk boundary.
-// Writes p (rank -> position), rank (position -> rank) and T to global scratch.
-__global__ void __launch_bounds__(kSortThreads2, 1)
-topw_sort_kernel(const float* __restrict__ delta, int32_t* __restrict__ p_out, int32_t* __restrict__ rank_out,
-                 int32_t* __restrict__ T_out, int N, int w) {
-  extern __shared__ __align__(16) unsigned char smraw[];
-  const int row = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nch = (N + kC - 1) / kC;
-  const int Np = pad32(N) + 32;
-  const int Npi = (Np + 7) & ~7;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smraw);                         // [Np]   (later: table)
-  uint16_t* idx = reinterpret_cast<uint16_t*>(keys + Np);                      // [Npi]  ping
-  uint16_t* idx2 = idx + Npi;                                                  // [Npi]  pong
-  uint16_t* cnt = idx2 + Npi;                                                  // [16][1024] (later: rank)
-  int32_t* wsum = reinterpret_cast<int32_t*>(cnt + 16 * kSortThreads2);        // [32]
-  __shared__ uint32_t red_and[kSortWarps2], red_or[kSortWarps2];
-
+// One CTA (L/2 threads) sorts segment blockIdx.x of row blockIdx.y ascending into skeys.
+template <int L>
+__global__ void __launch_bounds__(L / 2)
+topw_segsort_kernel(const float* __restrict__ delta, uint64_t* __restrict__ skeys, int N, int npad) {
+  __shared__ uint64_t sk[L];
+  const int seg = blockIdx.x, row = blockIdx.y, tid = threadIdx.x;
   const float* drow = delta + (size_t)row * N;
-  const int IT = (N + kSortThreads2 - 1) / kSortThreads2;
-  uint32_t kand = 0xffffffffu, kor = 0u;
-  {
-    float dv[kMaxItems];   // all loads first, then the stores
 #pragma unroll
-    for (int u = 0; u < kMaxItems; ++u) {
-      const int i = tid + u * kSortThreads2;
-      dv[u] = i < N ? drow[i] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kMaxItems; ++u) {
-      const int i = tid + u * kSortThreads2;
-      if (i < N) {
-        const uint32_t k = ~order_key(dv[u]);   // ascending k = delta descending
-        keys[pad32(i)] = k;
-        idx[pad32(i)] = (uint16_t)i;
-        kand &= k;
-        kor |= k;
-      }
-    }
+  for (int u = 0; u < 2; ++u) {
+    const int i = tid + u * (L / 2);
+    const int j = seg * L + i;
+    sk[i] = j < N ? topw_key(drow[j], j) : ~0ull;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kand &= __shfl_xor_sync(0xffffffffu, kand, o);
-    kor |= __shfl_xor_sync(0xffffffffu, kor, o);
-  }
-  if (lane == 0) { red_and[warp] = kand; red_or[warp] = kor; }
   __syncthreads();
-  uint32_t varying = 0;
-  {
-    uint32_t a = 0xffffffffu, o = 0u;
-    for (int i = 0; i < kSortWarps2; ++i) { a &= red_and[i]; o |= red_or[i]; }
-    varying = a ^ o;
+  for (int k = 2; k <= L; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      const int i = 2 * jj * (tid / jj) + (tid % jj);   // lower element of this thread's pair
+      const bool up = (i & k) == 0;
+      const uint64_t x = sk[i], y = sk[i + jj];
+      if ((x > y) == up) {
+        sk[i] = y;
+        sk[i + jj] = x;
+      }
+      __syncthreads();
+    }
   }
+  uint64_t* out = skeys + (size_t)row * npad + (size_t)seg * L;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) out[tid + u * (L / 2)] = sk[tid + u * (L / 2)];
+}
 
-  for (int shift = 0; shift < 32; shift += 4) {
-    if (((varying >> shift) & 0xFu) == 0) continue;   // every key has the same digit here
-    uint32_t kk[kMaxItems];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) cnt[c * kSortThreads2 + tid] = 0;
-#pragma unroll
-    for (int i = 0; i < kMaxItems; ++i) {
-      const int pos = tid * IT + i;
-      if (i < IT && pos < N) {
-        kk[i] = keys[pad32(pos)];
-        const uint32_t dg = (kk[i] >> shift) & 0xFu;
-        cnt[dg * kSortThreads2 + tid] += 1;
-      }
-    }
-    __syncthreads();
-    {  // exclusive scan of cnt in (digit, thread) order: 16 entries per thread
-      uint32_t v[16], sum = 0;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) { v[c] = cnt[tid * 16 + c]; sum += v[c]; }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) wsum[warp] = (int32_t)incl;
-      __syncthreads();
-      if (warp == 0) {
-        const uint32_t x = (uint32_t)wsum[lane];
-        uint32_t xi = x;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, xi, o);
-          if (lane >= o) xi += y;
-        }
-        wsum[lane] = (int32_t)(xi - x);
-      }
-      __syncthreads();
-      uint32_t run = (uint32_t)wsum[warp] + incl - sum;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) { cnt[tid * 16 + c] = (uint16_t)run; run += v[c]; }
-    }
-    __syncthreads();
-    // every read of `keys` in this pass happened before the barriers above, so items can be
-    // written as soon as their destinations are known; indices go to the other buffer
-#pragma unroll
-    for (int i = 0; i < kMaxItems; ++i) {
-      const int pos = tid * IT + i;
-      if (i < IT && pos < N) {
-        const uint32_t dg = (kk[i] >> shift) & 0xFu;
-        const int dst = cnt[dg * kSortThreads2 + tid];
-        cnt[dg * kSortThreads2 + tid] = (uint16_t)(dst + 1);
-        keys[pad32(dst)] = kk[i];
-        idx2[pad32(dst)] = idx[pad32(pos)];
-      }
-    }
-    __syncthreads();
-    uint16_t* t = idx; idx = idx2; idx2 = t;
-  }
-  // p[r] = idx[pad32(r)];  rank[j] in the counter area
-  uint16_t* rank = cnt;
+// Ranks of segment blockIdx.x of row blockIdx.y: rank[j] (position -> rank) and p[r] (rank ->
+// position).  The row's sorted segments are staged in shared memory.
+template <int L>
+__global__ void __launch_bounds__(L / 2)
+topw_rank_kernel(const uint64_t* __restrict__ skeys, int32_t* __restrict__ p_out, int32_t* __restrict__ rank_out,
+                 int N, int nseg) {
+  extern __shared__ __align__(16) uint64_t rk[];   // [nseg * L]
+  const int seg = blockIdx.x, row = blockIdx.y, tid = threadIdx.x;
+  const int npad = nseg * L;
+  const uint64_t* src = skeys + (size_t)row * npad;
+  for (int i = tid * 2; i < npad; i += L) *reinterpret_cast<uint4*>(rk + i) = *reinterpret_cast<const uint4*>(src + i);
+  __syncthreads();
   int32_t* prow = p_out + (size_t)row * N;
   int32_t* rrow = rank_out + (size_t)row * N;
-  for (int r = tid; r < N; r += kSortThreads2) {
-    const int j = idx[pad32(r)];
-    rank[j] = (uint16_t)r;
-    prow[r] = j;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = tid + u * (L / 2);
+    const uint64_t key = rk[seg * L + i];
+    const uint32_t j = (uint32_t)key;
+    if (j >= (uint32_t)N) continue;   // padding
+    int r = i;
+    for (int s2 = 0; s2 < nseg; ++s2) {
+      if (s2 == seg) continue;
+      const uint64_t* a = rk + s2 * L;
+      int lo = 0, n = L;                // lower bound: first index with a[] >= key (keys are distinct)
+      while (n > 0) {
+        const int half = n >> 1;
+        if (a[lo + half] < key) { lo += half + 1; n -= half + 1; }
+        else n = half;
+      }
+      r += lo;
+    }
     rrow[j] = r;
+    prow[r] = (int32_t)j;
   }
-  // thresholds: table[rb][k] = #positions < k*C whose rank is in bucket rb (u32, reuses keys)
-  uint32_t* table = keys;
-  const int cw = nch + 1;
-  for (int i = tid; i < nch * cw; i += kSortThreads2) table[i] = 0;
+}
+
+constexpr int kThThreads = 1024;
+constexpr int kThWarps = kThThreads / 32;
+
+// T_k = rank of the w-th best key among positions [0, kC) for every chunk boundary k (N when
+// kC <= w: nothing evicted yet), from a [rank bucket][position chunk] count table with prefix sums
+// over chunks.  One CTA per row.
+__global__ void __launch_bounds__(kThThreads)
+topw_thresh_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in, int32_t* __restrict__ T_out,
+                   int N, int w) {
+  extern __shared__ __align__(16) uint32_t table[];   // [nch][nch + 1]
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nch = (N + kC - 1) / kC, cw = nch + 1;
+  const int32_t* prow = p_in + (size_t)row * N;
+  const int32_t* rrow = rank_in + (size_t)row * N;
+  for (int i = tid; i < nch * cw; i += kThThreads) table[i] = 0;
   __syncthreads();
-  for (int j = tid; j < N; j += kSortThreads2) atomicAdd(&table[(rank[j] >> 7) * cw + (j >> 7)], 1u);
+  for (int j = tid; j < N; j += kThThreads) atomicAdd(&table[(rrow[j] >> 7) * cw + (j >> 7)], 1u);
   __syncthreads();
-  for (int rb = tid; rb < nch; rb += kSortThreads2) {
+  for (int rb = tid; rb < nch; rb += kThThreads) {
     uint32_t prev = 0;
     for (int k = 0; k <= nch; ++k) {
       const uint32_t t = table[rb * cw + k];
@@ -194,7 +153,7 @@ topw_sort_kernel(const float* __restrict__ delta, int32_t* __restrict__ p_out, i
     }
   }
   __syncthreads();
-  for (int k = warp; k <= nch; k += kSortWarps2) {
+  for (int k = warp; k <= nch; k += kThWarps) {
     const int Pk = min(k * kC, N);
     int Tk = N;
     if (Pk > w) {
@@ -220,7 +179,7 @@ topw_sort_kernel(const float* __restrict__ delta, int32_t* __restrict__ p_out, i
       int need = w - before;
       for (int r0 = rbs * 128; r0 < min(rbs * 128 + 128, N); r0 += 32) {
         const int r = r0 + lane;
-        const uint32_t m = __ballot_sync(0xffffffffu, r < N && (int)idx[pad32(min(r, N - 1))] < Pk);
+        const uint32_t m = __ballot_sync(0xffffffffu, r < N && prow[min(r, N - 1)] < Pk);
         const int c = __popc(m);
         if (c >= need) { Tk = r0 + nth_set_bit(m, need - 1); break; }
         need -= c;
@@ -365,19 +324,25 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
   int32_t* oje = pje + pbase;
   float* odl = pdl + pbase;
   int nfull[3] = {0, 0, 0}, npart[3] = {0, 0, 0};
+  // e_j and delta_j of this thread's 4 keys, loaded one round ahead
   int enext[4];
+  float dnext[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int j = tid * 4 + u;
     enext[u] = j < t1 ? erow[j] : 0;
+    dnext[u] = j < t1 ? drow[j] : 0.f;
   }
   for (int base = 0; base < t1; base += kListThreads * 4) {
     int ecur[4];
+    float dcur[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       ecur[u] = enext[u];
-      const int jn = base + kListThreads * 4 + tid * 4 + u;   // prefetch the next round
+      dcur[u] = dnext[u];
+      const int jn = base + kListThreads * 4 + tid * 4 + u;
       enext[u] = jn < t1 ? erow[jn] : 0;
+      dnext[u] = jn < t1 ? drow[jn] : 0.f;
     }
     int cf = 0, cq = 0;              // packed counts of this thread's full / partial keys
     uint32_t fbits = 0, qbits = 0;   // bit 3u + L: key u is full / partial in list L
@@ -436,7 +401,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
             out[L][of[L]] = j;
             if (L == 2) {
               oje[of[L]] = (j & 0xffff) | (ecur[u] << 16);
-              odl[of[L]] = drow[j] * kLog2e;
+              odl[of[L]] = dcur[u] * kLog2e;
             }
           }
           ++of[L];
@@ -596,19 +561,36 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
 
 }  // namespace
 
+template <int L>
+cudaError_t launch_topw_rank(const Plan& P, const float* delta, uint64_t* skeys, int32_t* pbuf, int32_t* rbuf,
+                             cudaStream_t s) {
+  const int rows = P.B * P.H;
+  const int nseg = (P.N + L - 1) / L;
+  topw_segsort_kernel<L><<<dim3(nseg, rows), L / 2, 0, s>>>(delta, skeys, P.N, nseg * L);
+  const int smem = nseg * L * (int)sizeof(uint64_t);
+  { cudaError_t ea = ensure_smem_limit(topw_rank_kernel<L>, smem); if (ea != cudaSuccess) return ea; }
+  topw_rank_kernel<L><<<dim3(nseg, rows), L / 2, smem, s>>>(skeys, pbuf, rbuf, P.N, nseg);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evict, void* ws,
                                 cudaStream_t s) {
   const int rows = P.B * P.H;
   const int nch = P.n_blocks;
-  const int Np = P.N + (P.N >> 5) + 32;
-  const size_t smem = (size_t)Np * 4 + (size_t)((Np + 7) & ~7) * 2 * 2 + 16 * kSortThreads2 * 2 + 32 * 4 +
-                      (size_t)(nch + 1) * 4;
-  if ((size_t)nch * (nch + 1) * 4 > (size_t)Np * 4) return cudaErrorInvalidValue;   // table must fit
-  { cudaError_t ea = ensure_smem_limit(topw_sort_kernel, (int)smem); if (ea != cudaSuccess) return ea; }
   int32_t* pbuf = ws_ptr<int32_t>(ws, P.off_tw_p);
   int32_t* rbuf = ws_ptr<int32_t>(ws, P.off_tw_rank);
   int32_t* Tbuf = ws_ptr<int32_t>(ws, P.off_tw_T);
-  topw_sort_kernel<<<rows, kSortThreads2, smem, s>>>(delta, pbuf, rbuf, Tbuf, P.N, P.w);
+  uint64_t* skeys = ws_ptr<uint64_t>(ws, P.off_tw_keys);
+  cudaError_t e;
+  switch (topw_seg_len(P.N)) {
+    case 512: e = launch_topw_rank<512>(P, delta, skeys, pbuf, rbuf, s); break;
+    case 1024: e = launch_topw_rank<1024>(P, delta, skeys, pbuf, rbuf, s); break;
+    default: e = launch_topw_rank<2048>(P, delta, skeys, pbuf, rbuf, s); break;
+  }
+  if (e != cudaSuccess) return e;
+  const int tsmem = nch * (nch + 1) * (int)sizeof(uint32_t);
+  { cudaError_t ea = ensure_smem_limit(topw_thresh_kernel, tsmem); if (ea != cudaSuccess) return ea; }
+  topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w);
   topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
   topw_lists_kernel<<<dim3(P.n_pairs, rows), kListThreads, 0, s>>>(
