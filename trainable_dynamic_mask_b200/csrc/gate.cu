@@ -295,21 +295,43 @@ gate_fwd_mma_kernel(const uint16_t* __restrict__ V, const uint16_t* __restrict__
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dch = d / 8;
   // ---- stage V (16 positions x K) and Delta (K x H, padded to 8 HT columns)
-  for (int q = tid; q < kGmP * KC; q += kGmThreads) {
-    const int p = q / KC, kc = q % KC;
-    const int g = kc / dch, c = kc % dch;
-    const int pos = p0 + p;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (pos < N) v = *reinterpret_cast<const uint4*>(V + ((size_t)(b * Hkv + g) * N + pos) * d + c * 8);
-    *reinterpret_cast<uint4*>(Vs + (size_t)p * K + ((kc ^ (p & 7)) * 8)) = v;
+  // batches of kGmBatch 16-byte loads per thread, all issued before their stores
+  constexpr int kGmBatch = 8;
+  for (int q0 = 0; q0 < kGmP * KC; q0 += kGmBatch * kGmThreads) {
+    uint4 v[kGmBatch];
+#pragma unroll
+    for (int u = 0; u < kGmBatch; ++u) {
+      const int q = q0 + u * kGmThreads + tid;
+      const int p = q / KC, kc = q % KC;
+      const int g = kc / dch, c = kc % dch;
+      const int pos = p0 + p;
+      v[u] = make_uint4(0, 0, 0, 0);
+      if (q < kGmP * KC && pos < N) v[u] = *reinterpret_cast<const uint4*>(V + ((size_t)(b * Hkv + g) * N + pos) * d + c * 8);
+    }
+#pragma unroll
+    for (int u = 0; u < kGmBatch; ++u) {
+      const int q = q0 + u * kGmThreads + tid;
+      const int p = q / KC, kc = q % KC;
+      if (q < kGmP * KC) *reinterpret_cast<uint4*>(Vs + (size_t)p * K + ((kc ^ (p & 7)) * 8)) = v[u];
+    }
   }
   if ((H & 7) == 0) {
     const int hc = H / 8;
-    for (int q = tid; q < K * HT; q += kGmThreads) {
-      const int r = q / HT, c = q % HT;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (c < hc) v = *reinterpret_cast<const uint4*>(Delta + (size_t)r * H + c * 8);
-      *reinterpret_cast<uint4*>(Ds + (size_t)r * 8 * HT + c * 8) = v;
+    for (int q0 = 0; q0 < K * HT; q0 += kGmBatch * kGmThreads) {
+      uint4 v[kGmBatch];
+#pragma unroll
+      for (int u = 0; u < kGmBatch; ++u) {
+        const int q = q0 + u * kGmThreads + tid;
+        const int r = q / HT, c = q % HT;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (q < K * HT && c < hc) v[u] = *reinterpret_cast<const uint4*>(Delta + (size_t)r * H + c * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < kGmBatch; ++u) {
+        const int q = q0 + u * kGmThreads + tid;
+        const int r = q / HT, c = q % HT;
+        if (q < K * HT) *reinterpret_cast<uint4*>(Ds + (size_t)r * 8 * HT + c * 8) = v[u];
+      }
     }
   } else {
     for (int q = tid; q < K * 8 * HT; q += kGmThreads) {

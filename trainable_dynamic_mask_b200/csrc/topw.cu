@@ -26,6 +26,8 @@
 //     pair: full keys (selected by every existing row of the range: j <= t0 and e_j >= t1) first,
 //     then the partial ones (keys evicted inside the range and the range's own keys), each in
 //     ascending order.
+#include <limits.h>
+
 #include "common.cuh"
 
 namespace dma {
@@ -90,22 +92,27 @@ topw_segsort_kernel(const float* __restrict__ delta, uint64_t* __restrict__ skey
 }
 
 // Ranks of segment blockIdx.x of row blockIdx.y: rank[j] (position -> rank) and p[r] (rank ->
-// position).  The row's sorted segments are staged in shared memory.
+// position).  The row's sorted segments are staged in shared memory; one key per thread (two for
+// L = 2048).
 template <int L>
-__global__ void __launch_bounds__(L / 2)
+constexpr int rank_threads() { return L < 1024 ? L : 1024; }
+
+template <int L>
+__global__ void __launch_bounds__(rank_threads<L>())
 topw_rank_kernel(const uint64_t* __restrict__ skeys, int32_t* __restrict__ p_out, int32_t* __restrict__ rank_out,
                  int N, int nseg) {
+  constexpr int kT = rank_threads<L>();
   extern __shared__ __align__(16) uint64_t rk[];   // [nseg * L]
   const int seg = blockIdx.x, row = blockIdx.y, tid = threadIdx.x;
   const int npad = nseg * L;
   const uint64_t* src = skeys + (size_t)row * npad;
-  for (int i = tid * 2; i < npad; i += L) *reinterpret_cast<uint4*>(rk + i) = *reinterpret_cast<const uint4*>(src + i);
+  for (int i = tid * 2; i < npad; i += 2 * kT) *reinterpret_cast<uint4*>(rk + i) = *reinterpret_cast<const uint4*>(src + i);
   __syncthreads();
   int32_t* prow = p_out + (size_t)row * N;
   int32_t* rrow = rank_out + (size_t)row * N;
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int i = tid + u * (L / 2);
+  for (int u = 0; u < L / kT; ++u) {
+    const int i = tid + u * kT;
     const uint64_t key = rk[seg * L + i];
     const uint32_t j = (uint32_t)key;
     if (j >= (uint32_t)N) continue;   // padding
@@ -113,12 +120,11 @@ topw_rank_kernel(const uint64_t* __restrict__ skeys, int32_t* __restrict__ p_out
     for (int s2 = 0; s2 < nseg; ++s2) {
       if (s2 == seg) continue;
       const uint64_t* a = rk + s2 * L;
-      int lo = 0, n = L;                // lower bound: first index with a[] >= key (keys are distinct)
-      while (n > 0) {
-        const int half = n >> 1;
-        if (a[lo + half] < key) { lo += half + 1; n -= half + 1; }
-        else n = half;
-      }
+      int lo = 0;                       // lower bound: first index with a[] >= key (keys are distinct)
+#pragma unroll
+      for (int step = L / 2; step > 0; step >>= 1)
+        if (a[lo + step - 1] < key) lo += step;
+      lo += a[lo] < key ? 1 : 0;
       r += lo;
     }
     rrow[j] = r;
@@ -202,9 +208,11 @@ __global__ void __launch_bounds__(kEvThreads)
 topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in,
                   const int32_t* __restrict__ T_in, int32_t* __restrict__ evict, int32_t* __restrict__ status,
                   int N, int w) {
+  constexpr int kEvU = 4;            // ranks scanned per thread per round
   __shared__ int32_t crank[kC];      // ranks of the chunk's own keys
   __shared__ int32_t L[kC];          // old candidates, ascending rank
-  __shared__ int32_t wcount[kEvThreads / 32];
+  __shared__ int32_t Lpos[kC];       // their positions
+  __shared__ int32_t wcount[kEvU][kEvThreads / 32];
   const int k = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = (N + kC - 1) / kC;
@@ -216,23 +224,41 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   const int Ta = T[k], Tb = T[k + 1], Tf = T[nch];
   const int Sk = min(t0, w);
   if (tid < t1 - t0) crank[tid] = rrow[t0 + tid];
-  // old candidates in rank order
+  // old candidates in rank order: the ranks in (Tb, Ta] held by positions < t0; all loads of a round
+  // are issued before its ballots
   int nL = 0;
   const int rhi = min(Ta, N - 1);
-  for (int r0 = Tb + 1; r0 <= rhi; r0 += kEvThreads) {
-    const int r = r0 + tid;
-    const bool in = r <= rhi && prow[r] < t0;
-    const uint32_t m = __ballot_sync(0xffffffffu, in);
-    if (lane == 0) wcount[warp] = __popc(m);
-    __syncthreads();
-    int before = nL, total = 0;
-    for (int i = 0; i < kEvThreads / 32; ++i) {
-      if (i < warp) before += wcount[i];
-      total += wcount[i];
+  for (int r0 = Tb + 1; r0 <= rhi; r0 += kEvThreads * kEvU) {
+    int pos[kEvU];
+#pragma unroll
+    for (int u = 0; u < kEvU; ++u) {
+      const int r = r0 + u * kEvThreads + tid;
+      pos[u] = r <= rhi ? prow[r] : INT_MAX;
     }
-    if (in) {
-      const int slot = before + __popc(m & lanemask_lt());
-      if (slot < kC) L[slot] = r;
+    uint32_t m[kEvU];
+#pragma unroll
+    for (int u = 0; u < kEvU; ++u) {
+      m[u] = __ballot_sync(0xffffffffu, pos[u] < t0);
+      if (lane == 0) wcount[u][warp] = __popc(m[u]);
+    }
+    __syncthreads();
+    int before = nL;   // candidates at ranks before this thread's first one (rank order = u, warp, lane)
+    int total = 0;
+#pragma unroll
+    for (int u = 0; u < kEvU; ++u) {
+      int bu = 0, tu = 0;
+      for (int i = 0; i < kEvThreads / 32; ++i) {
+        if (i < warp) bu += wcount[u][i];
+        tu += wcount[u][i];
+      }
+      if (pos[u] < t0) {
+        const int slot = before + total + bu + __popc(m[u] & lanemask_lt());
+        if (slot < kC) {
+          L[slot] = r0 + u * kEvThreads + tid;
+          Lpos[slot] = pos[u];
+        }
+      }
+      total += tu;
     }
     nL += total;
     __syncthreads();
@@ -242,13 +268,31 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
     nL = kC;
   }
   __syncthreads();
+  // The chunk's keys in rank order, and pmask[q] = offsets (t - t0) of the chunk's q best keys:
+  // the chunk keys better than rank r are pmask[#{chunk ranks < r}].
+  __shared__ int32_t srank[kC];
+  __shared__ uint32_t pmask[kC + 1][kEvThreads / 32];
+  const int nc = t1 - t0;
+  int cr = kC;   // rank of offset tid among the chunk's keys
+  if (tid < nc) {
+    const int my = crank[tid];
+    int q = 0;
+    for (int i = 0; i < nc; ++i) q += crank[i] < my;
+    cr = q;
+    srank[q] = my;
+  }
+  for (int q = 0; q <= nc; ++q) {
+    const uint32_t m = __ballot_sync(0xffffffffu, cr < q);   // word `warp`: offsets 32 warp + lane
+    if (lane == 0) pmask[q][warp] = m;
+  }
+  __syncthreads();
   const int ncand = nL + (t1 - t0);
   for (int c = tid; c < ncand; c += kEvThreads) {
     int r, j, base, e = -1;
     bool scan = false;
     if (c < nL) {
       r = L[c];
-      j = prow[r];
+      j = Lpos[c];
       base = Sk - (nL - c);
       scan = true;
     } else {
@@ -260,18 +304,37 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
       } else if (Ta < N && r > Ta) {
         e = j;                         // never selected
       } else {
-        int above = 0;                 // old members with rank in (r, Ta]
-        for (int i = 0; i < nL; ++i) above += L[i] > r;
-        base = Sk - above;
+        int lo = 0, n = nL;            // old members with rank in (r, Ta]: L is ascending
+        while (n > 0) {
+          const int half = n >> 1;
+          if (L[lo + half] <= r) { lo += half + 1; n -= half + 1; }
+          else n = half;
+        }
+        base = Sk - (nL - lo);
         if (base >= w) e = j;
         else scan = true;
       }
     }
     if (scan) {
-      int count = base;
+      // e = the chunk position at which the count of keys better than r, starting from base,
+      // reaches w: the (w - base)-th chunk key better than r in position order
+      int lo = 0, n = nc;
+      while (n > 0) {
+        const int half = n >> 1;
+        if (srank[lo + half] < r) { lo += half + 1; n -= half + 1; }
+        else n = half;
+      }
+      int left = w - base;
       e = -2;
-      for (int t = t0; t < t1; ++t) {
-        if (crank[t - t0] < r && ++count >= w) { e = max(j, t); break; }
+#pragma unroll
+      for (int wd = 0; wd < kEvThreads / 32; ++wd) {
+        const uint32_t m = pmask[lo][wd];
+        const int cnt = __popc(m);
+        if (cnt >= left) {
+          e = max(j, t0 + 32 * wd + nth_set_bit(m, left - 1));
+          break;
+        }
+        left -= cnt;
       }
       if (e == -2) {                   // cannot happen: such keys are evicted inside the chunk
         e = t1;
@@ -353,12 +416,19 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
 #pragma unroll
       for (int L = 0; L < 3; ++L) {
         const bool valid = L != 1 || has_b;
-        const bool live = valid && j < hi[L] && e > max(j, lo[L]);
-        const bool full = live && j <= lo[L] && e >= hi[L];
+        bool full, part;
+        if (j <= t0) {   // j <= every range's first row: live iff e > lo, full iff e >= hi
+          full = valid && e >= hi[L];
+          part = valid && e > lo[L] && e < hi[L];
+        } else {
+          const bool live = valid && j < hi[L] && e > max(j, lo[L]);
+          full = live && j <= lo[L] && e >= hi[L];
+          part = live && !full;
+        }
         fbits |= (uint32_t)full << (3 * u + L);
-        qbits |= (uint32_t)(live && !full) << (3 * u + L);
+        qbits |= (uint32_t)part << (3 * u + L);
         cf += (int)full << (kListBits * L);
-        cq += (int)(live && !full) << (kListBits * L);
+        cq += (int)part << (kListBits * L);
       }
     }
     int incf = cf, incq = cq;
@@ -569,7 +639,7 @@ cudaError_t launch_topw_rank(const Plan& P, const float* delta, uint64_t* skeys,
   topw_segsort_kernel<L><<<dim3(nseg, rows), L / 2, 0, s>>>(delta, skeys, P.N, nseg * L);
   const int smem = nseg * L * (int)sizeof(uint64_t);
   { cudaError_t ea = ensure_smem_limit(topw_rank_kernel<L>, smem); if (ea != cudaSuccess) return ea; }
-  topw_rank_kernel<L><<<dim3(nseg, rows), L / 2, smem, s>>>(skeys, pbuf, rbuf, P.N, nseg);
+  topw_rank_kernel<L><<<dim3(nseg, rows), rank_threads<L>(), smem, s>>>(skeys, pbuf, rbuf, P.N, nseg);
   return cudaGetLastError();
 }
 
