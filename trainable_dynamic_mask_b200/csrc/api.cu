@@ -51,6 +51,55 @@ cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
   return e;
 }
 
+// Work units of the attention forward (see FwdSchedule).  The split counts depend only on the
+// problem's shape and a fixed reference of 148 SMs, so that the workspace plan and the launch agree.
+// Splitting costs a second pipeline start and a merge per split pair, so pairs are split only when
+// there are fewer pairs than SMs: then each pair gets S = min(4, ceil(SMs / pairs), its tiles)
+// splits (its list length estimated as min(t1, min(w, N) + 128) keys).
+void fwd_schedule(const Plan& P, FwdSchedule* S) {
+  constexpr int kRefSMs = 148;
+  const int BH = P.B * P.H;
+  const int minwn = P.w < P.N ? P.w : P.N;
+  const long items = (long)BH * P.n_pairs;
+  const long want = items >= kRefSMs ? 1 : (kRefSMs + items - 1) / items;
+  int est[kMaxPairs], split[kMaxPairs], order[kMaxPairs];
+  for (int kp = 0; kp < P.n_pairs; ++kp) {
+    const int t1 = (kp + 1) * kPairQ < P.N ? (kp + 1) * kPairQ : P.N;
+    const int live = t1 < minwn + kBlockQ ? t1 : minwn + kBlockQ;
+    est[kp] = (live + kBlockQ - 1) / kBlockQ;
+    long sp = want < kMaxSplits ? want : kMaxSplits;
+    if (sp > est[kp]) sp = est[kp];
+    split[kp] = (int)(sp < 1 ? 1 : sp);
+    order[kp] = kp;
+  }
+  // heaviest units first: cost est / S, ties to the later pair
+  for (int a = 1; a < P.n_pairs; ++a)
+    for (int b = a; b > 0; --b) {
+      const int x = order[b - 1], y = order[b];
+      if ((long)est[y] * split[x] > (long)est[x] * split[y] ||
+          ((long)est[y] * split[x] == (long)est[x] * split[y] && y > x)) {
+        order[b - 1] = y;
+        order[b] = x;
+      } else {
+        break;
+      }
+    }
+  memset(S, 0, sizeof(*S));
+  int start = 0, slot = 0;
+  for (int i = 0; i < P.n_pairs; ++i) {
+    const int kp = order[i];
+    S->g[i].kp = kp;
+    S->g[i].S = split[kp];
+    S->g[i].start = start;
+    S->g[i].slot = split[kp] > 1 ? slot : -1;
+    start += BH * split[kp];
+    if (split[kp] > 1) slot += BH * split[kp];
+  }
+  S->n_groups = P.n_pairs;
+  S->n_units = start;
+  S->n_slots = slot;
+}
+
 dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   if (p == nullptr || P == nullptr) return DMA_ERR_INVALID_ARG;
   if (p->B < 1 || p->H < 1 || p->Hkv < 1 || p->N < 1 || p->Nq < 1 || p->d < 1 || p->w < 1)
@@ -99,8 +148,12 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_lists = take(BH * R.n_blocks * (size_t)R.list_cap * sizeof(int32_t));
     R.off_pcounts = take(BH * R.n_pairs * 2 * sizeof(int32_t));
     R.off_plists = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(int32_t));
-    R.off_pje = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(int32_t));
+    R.off_plen = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(int32_t));
     R.off_pdl = take(BH * R.n_pairs * (size_t)R.pair_cap * sizeof(float));
+    fwd_schedule(R, &R.sched);
+    R.off_fpart = take((size_t)R.sched.n_slots * 2 * R.d * kBlockQ * sizeof(float));
+    R.off_fml = take((size_t)R.sched.n_slots * 2 * 2 * kBlockQ * sizeof(float));
+    R.off_fcnt = take(BH * R.n_pairs * 4 * sizeof(int32_t));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));

@@ -8,8 +8,10 @@
 // Work item = (b, h, pair of query blocks: 256 rows), walking the pair's live-key list (the union
 // of the two blocks' lists; full keys first) in tiles of 128 keys.  Each gathered K/V tile feeds
 // both 128-row halves, so the gather traffic per tensor-core FLOP is half that of 128-row items.
-// The kernel is persistent: one CTA per SM walks items heaviest-first (snake order over the CTAs),
-// and the next item's Q and first tiles load while the current one finishes.
+// The kernel is persistent: one CTA per SM walks work units heaviest-first (snake order over the
+// CTAs), and the next unit's Q and first tiles load while the current one finishes.  A unit is a
+// pair, or one of S splits of a long pair's list: the split that finishes last merges the others'
+// partial (O, m, l) with its own, so that few heavy pairs still spread evenly over the SMs.
 //
 // Warp roles (512 threads):
 //   warps 0-3  softmax of query half 0, warps 4-7 softmax of half 1: thread r owns query row r of
@@ -24,7 +26,7 @@
 //              swizzled, the layout the MMA reads).  One warp's TMA issue rate caps its gather
 //              throughput, so seven warps issue.
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D); P_h aliases S_h.
-// Stages: Q 1 (both halves), K 2, V 2.  Tile metadata (delta_j log2(e), j | e_j << 16) is read by
+// Stages: Q 1 (both halves), K 2, V 2.  Tile metadata (delta_j log2(e), j, e_j - j) is read by
 // the softmax threads straight from the list, one entry per thread, through a shared buffer.
 // Every wait is bounded (tc::mbar_wait) and reports a timeout through the workspace status word;
 // every TMEM load/store (warp-collective) sits behind warp-uniform decisions.
@@ -41,8 +43,8 @@ namespace {
 
 constexpr int kTcThreads = 512;
 constexpr int kMmaWarp = 8;
-constexpr int kVWarp0 = 9, kVWarps = 3;     // V producers: row groups 11 + 11 + 10
-constexpr int kKWarp0 = 12, kKWarps = 4;    // Q/K producers: row groups 8 per warp
+constexpr int kVWarp0 = 9;                  // V producers: warps 9-11, row groups 11 + 11 + 10
+constexpr int kKWarp0 = 12;                 // Q/K producers: warps 12-15, row groups 8 per warp
 // Register split (setmaxnreg): launched with 128 per thread (512 x 128 = 65536), warpgroups 2 and 3
 // give back to 48 and the softmax warpgroups take 208: 256 x 48 + 256 x 208 = 65536.
 constexpr int kRegsSoftmax = 208, kRegsOther = 48;
@@ -53,7 +55,7 @@ constexpr int kPolyEvery = 4;               // one pair in kPolyEvery takes the 
 
 enum : int { kErrTimeoutQ = 0x100, kErrTimeoutK = 0x200, kErrTimeoutS = 0x400, kErrTimeoutP = 0x800,
              kErrTimeoutPV = 0x1000, kErrTimeoutKEmpty = 0x2000, kErrTimeoutV = 0x4000,
-             kErrTimeoutVEmpty = 0x8000, kErrTimeoutQEmpty = 0x10000, kErrSmemAlign = 0x40000 };
+             kErrTimeoutVEmpty = 0x8000, kErrTimeoutQEmpty = 0x10000, kErrTimeoutMerge = 0x20000, kErrSmemAlign = 0x40000 };
 
 template <int D>
 struct TcSmem {
@@ -62,8 +64,8 @@ struct TcSmem {
   static constexpr int kQ = 0;                        // [2 query halves]
   static constexpr int kK = kQ + 2 * kTile;           // [kKStages]
   static constexpr int kV = kK + kKStages * kTile;    // [kVStages]
-  static constexpr int kMeta = kV + kVStages * kTile; // [2 halves][2 buffers][dl f32 | je i32][128]
-  static constexpr int kBars = kMeta + 2 * 2 * 2 * kTcBK * 4;
+  static constexpr int kMeta = kV + kVStages * kTile; // [2 halves][2 buffers][dl f32 | j | e - j][128]
+  static constexpr int kBars = kMeta + 2 * 2 * 3 * kTcBK * 4;
   static constexpr int kBytes = kBars + 512;
 };
 
@@ -75,6 +77,7 @@ struct TcBars {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  int merge_old[2];   // per softmax warpgroup: arrivals seen by its unit's merge counter
 };
 
 DMA_DEVINL void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
@@ -94,14 +97,6 @@ DMA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r
       "%3, %4, %5, %6}], [%7];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
       : "memory");
-}
-
-DMA_DEVINL void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
 // Warp-uniform bounded wait (every lane of the warp calls it).
@@ -241,26 +236,61 @@ DMA_DEVINL void issue_pv(uint32_t tmem, int half, uint64_t dv, bool first, uint6
   tc::commit(done);
 }
 
-// Item q of the heaviest-first order: pair kp (late pairs have the longest lists), row bh.
-struct Item { int bh, kp; };
-DMA_DEVINL Item item_of(int q, int BH, int n_pairs) { return Item{q % BH, n_pairs - 1 - q / BH}; }
-// The r-th item of CTA c among G: snake order over the CTAs, so that the CTAs that took the heavier
-// items of one round take the lighter ones of the next.
-DMA_DEVINL int item_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+// 32 consecutive outputs of a row (16-byte stores).
+DMA_DEVINL void store_row32(uint16_t* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 32; u += 8) {
+    uint4 w;
+    w.x = pack_bf16x2(v[u], v[u + 1]);
+    w.y = pack_bf16x2(v[u + 2], v[u + 3]);
+    w.z = pack_bf16x2(v[u + 4], v[u + 5]);
+    w.w = pack_bf16x2(v[u + 6], v[u + 7]);
+    *reinterpret_cast<uint4*>(dst + u) = w;
+  }
+}
+DMA_DEVINL void store_row32(float* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
+}
+DMA_DEVINL int ld_acquire(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Work unit u (see FwdSchedule): pair kp of row bh, split s of S (its list's tiles
+// [s n / S, (s + 1) n / S)), partial-result slot (-1 when the pair is not split).
+struct Unit { int bh, kp, s, S, slot; };
+DMA_DEVINL Unit unit_of(const FwdSchedule& sc, int u) {
+  int g = 0;
+  while (g + 1 < sc.n_groups && u >= sc.g[g + 1].start) ++g;
+  const int idx = u - sc.g[g].start, S = sc.g[g].S;
+  return Unit{idx / S, sc.g[g].kp, idx % S, S, S > 1 ? sc.g[g].slot + idx : -1};
+}
+// The r-th unit of CTA c among G: snake order over the CTAs, so that the CTAs that took the heavier
+// units of one round take the lighter ones of the next.
+DMA_DEVINL int unit_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+// Tiles [tb, te) of the unit's pair list of n_live entries.
+DMA_DEVINL void unit_tiles(const Unit& x, int n_live, int& tb, int& te) {
+  const int n = (n_live + kTcBK - 1) / kTcBK;
+  tb = x.s * n / x.S;
+  te = (x.s + 1) * n / x.S;
+}
 
 template <int D, typename OutT>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, const int32_t* __restrict__ pcounts,
-                   const int32_t* __restrict__ plists, const int32_t* __restrict__ pje,
-                   const float* __restrict__ pdl, OutT* __restrict__ O, float* __restrict__ LSE,
-                   int32_t* __restrict__ status, int BH, int H, int G, int N, int n_pairs, int pair_cap,
-                   float scale_log2) {
+                   const __grid_constant__ CUtensorMap vmap, const __grid_constant__ FwdSchedule sched,
+                   const int32_t* __restrict__ pcounts, const int32_t* __restrict__ plists,
+                   const int32_t* __restrict__ plen, const float* __restrict__ pdl, OutT* __restrict__ O,
+                   float* __restrict__ LSE, float* __restrict__ fpart, float* __restrict__ fml,
+                   int32_t* __restrict__ fcnt, int32_t* __restrict__ status, int H, int G, int N, int n_pairs,
+                   int pair_cap, float scale_log2) {
   using S = TcSmem<D>;
   extern __shared__ __align__(1024) unsigned char sm[];
   TcBars& bar = *reinterpret_cast<TcBars*>(sm + S::kBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_items = BH * n_pairs;
+  const int n_units = sched.n_units;
   const int cta = blockIdx.x, n_ctas = gridDim.x;
   volatile int* abort_flag = &bar.abort_flag;
 
@@ -318,17 +348,18 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       int n_done = 0;              // items done (Q buffer phase)
       bool ok = !*abort_flag;
       for (int r = 0; ok; ++r) {
-        const int q = item_index(r, cta, n_ctas);
-        if (q >= n_items) break;
-        const Item it = item_of(q, BH, n_pairs);
+        const int u = unit_index(r, cta, n_ctas);
+        if (u >= n_units) break;
+        const Unit it = unit_of(sched, u);
         const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap;
-        const int n_live = pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1];
-        const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+        int tb, te;
+        unit_tiles(it, pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1], tb, te);
+        const int n_tiles = te - tb;
         const int t0 = it.kp * 256;
         const int b = it.bh / H, h = it.bh % H, g = h / G, Hkv = H / G;
         const int kvrow0 = (b * Hkv + g) * N;
-        if (n_tiles == 0) continue;   // cannot happen: every query row selects at least one key
-        const int32_t* list = plists + lbase + 4 * grp;
+        if (n_tiles == 0) continue;   // an empty split: nothing to load
+        const int32_t* list = plists + lbase + (size_t)tb * kTcBK + 4 * grp;
         int4 jn = make_int4(0, 0, 0, 0);
         if (issuer) jn = *reinterpret_cast<const int4*>(list);
         if (kside) {
@@ -386,11 +417,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         int n_done = 0;            // items done
         bool ok = !*abort_flag;
         for (int r = 0; ok; ++r) {
-          const int q = item_index(r, cta, n_ctas);
-          if (q >= n_items) break;
-          const Item it = item_of(q, BH, n_pairs);
-          const int n_live = pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1];
-          const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
+          const int u = unit_index(r, cta, n_ctas);
+          if (u >= n_units) break;
+          const Unit it = unit_of(sched, u);
+          int tb, te;
+          unit_tiles(it, pcounts[((size_t)it.bh * n_pairs + it.kp) * 2 + 1], tb, te);
+          const int n_tiles = te - tb;
           if (n_tiles == 0) continue;
           if (!(ok = tc::mbar_wait(&bar.q_full, n_done & 1, abort_flag, status, kErrTimeoutQ))) break;
           // first K tile: both halves
@@ -452,22 +484,24 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     const int r = tid & 127;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + h * 128 + lane_base, tO = tmem + 256 + h * 128 + lane_base;
-    float* meta = reinterpret_cast<float*>(sm + S::kMeta) + h * 2 * 2 * kTcBK;   // [2 buffers][dl | je][128]
+    float* meta = reinterpret_cast<float*>(sm + S::kMeta) + h * 2 * 3 * kTcBK;   // [2 buffers][dl | j | len][128]
     const uint64_t sc2 = f2(scale_log2, scale_log2);
     int tcount = 0;
     bool ok = !*abort_flag;
     for (int rr = 0; ok; ++rr) {
-      const int q = item_index(rr, cta, n_ctas);
-      if (q >= n_items) break;
-      const Item it = item_of(q, BH, n_pairs);
+      const int u = unit_index(rr, cta, n_ctas);
+      if (u >= n_units) break;
+      const Unit it = unit_of(sched, u);
       const int32_t* cnt = pcounts + ((size_t)it.bh * n_pairs + it.kp) * 2;
-      const int n_full = cnt[0], n_live = cnt[1];
-      const int n_tiles = (n_live + kTcBK - 1) / kTcBK;
-      if (n_tiles == 0) continue;
-      const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap;
+      const int n_full = cnt[0];
+      int tb, te;
+      unit_tiles(it, cnt[1], tb, te);
+      const int n_tiles = te - tb;
+      const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap + (size_t)tb * kTcBK;
       const int t = it.kp * 256 + h * 128 + r;   // this thread's query row
-      float dl_n = pdl[lbase + r];
-      int je_n = pje[lbase + r];
+      float dl_n = n_tiles > 0 ? pdl[lbase + r] : 0.f;
+      int jj_n = n_tiles > 0 ? plists[lbase + r] : -1;
+      int ln_n = n_tiles > 0 ? plen[lbase + r] : 0;
       float m_used = -INFINITY, l = 0.f;
       for (int i = 0; i < n_tiles; ++i) {
         const int tt = tcount + i;
@@ -480,17 +514,19 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 #pragma unroll
         for (int c = 0; c < kTcBK / 32; ++c) tc::tmem_ld32(tS + c * 32, sr[c]);
         // this tile's metadata: entry r from this thread, the others through the shared buffer
-        float* buf = meta + (i & 1) * 2 * kTcBK;
+        float* buf = meta + (i & 1) * 3 * kTcBK;
         buf[r] = dl_n;
-        reinterpret_cast<int32_t*>(buf)[kTcBK + r] = je_n;
+        reinterpret_cast<int32_t*>(buf)[kTcBK + r] = jj_n;
+        reinterpret_cast<int32_t*>(buf)[2 * kTcBK + r] = ln_n;
         if (i + 1 < n_tiles) {
           dl_n = pdl[lbase + (i + 1) * kTcBK + r];
-          je_n = pje[lbase + (i + 1) * kTcBK + r];
+          jj_n = plists[lbase + (i + 1) * kTcBK + r];
+          ln_n = plen[lbase + (i + 1) * kTcBK + r];
         }
         group_sync(h);
         tc::tmem_wait_ld();
         const float4* dl4 = reinterpret_cast<const float4*>(buf);
-        const bool full_tile = (i + 1) * kTcBK <= n_full;
+        const bool full_tile = (tb + i + 1) * kTcBK <= n_full;
         float mt = -INFINITY;
         if (full_tile) {
 #pragma unroll
@@ -511,11 +547,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             s4[3] = __float_as_uint(v3);
           }
         } else {
-          const int4* je4 = reinterpret_cast<const int4*>(buf + kTcBK);
+          // key j is selected by rows t in [j, j + len): (unsigned)(t - j) < len
+          const int4* jj4 = reinterpret_cast<const int4*>(buf + kTcBK);
+          const int4* ln4 = reinterpret_cast<const int4*>(buf + 2 * kTcBK);
 #pragma unroll
           for (int c4 = 0; c4 < kTcBK / 4; ++c4) {
             const float4 d = dl4[c4];
-            const int4 w = je4[c4];
+            const int4 jv = jj4[c4], lv = ln4[c4];
             const int c = 4 * c4;
             uint32_t* s4 = &sr[c / 32][c % 32];
             const uint64_t va = f2_fma(f2(__uint_as_float(s4[0]), __uint_as_float(s4[1])), sc2, f2(d.x, d.y));
@@ -523,13 +561,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             float v[4];
             f2_split(va, v[0], v[1]);
             f2_split(vb, v[2], v[3]);
-            const int ww[4] = {w.x, w.y, w.z, w.w};
+            v[0] = (uint32_t)(t - jv.x) < (uint32_t)lv.x ? v[0] : -INFINITY;
+            v[1] = (uint32_t)(t - jv.y) < (uint32_t)lv.y ? v[1] : -INFINITY;
+            v[2] = (uint32_t)(t - jv.z) < (uint32_t)lv.z ? v[2] : -INFINITY;
+            v[3] = (uint32_t)(t - jv.w) < (uint32_t)lv.w ? v[3] : -INFINITY;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int jj = (ww[u] << 16) >> 16, ee = ww[u] >> 16;   // key (-1: padding), e_j
-              v[u] = (jj <= t && t < ee) ? v[u] : -INFINITY;
-              s4[u] = __float_as_uint(v[u]);
-            }
+            for (int u = 0; u < 4; ++u) s4[u] = __float_as_uint(v[u]);
             mt = max3(mt, v[0], v[1]);
             mt = max3(mt, v[2], v[3]);
           }
@@ -590,41 +627,112 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
       if (!ok) break;
       // ---- epilogue: O row = O_h / l, LSE = (m + log2 l) ln 2
-      const int last = tcount + n_tiles - 1;
-      if (!wait_all(&bar.pv_done[h], last & 1, abort_flag, status, kErrTimeoutPV)) {
-        ok = false;
-        break;
+      const bool own = n_tiles > 0;
+      if (own) {
+        const int last = tcount + n_tiles - 1;
+        if (!wait_all(&bar.pv_done[h], last & 1, abort_flag, status, kErrTimeoutPV)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after();
       }
-      tc::fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
       const bool valid = t < N;
       OutT* orow = O + ((size_t)it.bh * N + (valid ? t : 0)) * D;
+      if (it.S == 1) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tc::tmem_ld32(tO + c * 32, ov);
-        tc::tmem_wait_ld();
-        if (valid) {
-          if constexpr (sizeof(OutT) == 2) {
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tO + c * 32, ov);
+          tc::tmem_wait_ld();
+          float of[32];
 #pragma unroll
-            for (int u = 0; u < 32; u += 8) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(ov[u]) * inv, __uint_as_float(ov[u + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(ov[u + 2]) * inv, __uint_as_float(ov[u + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(ov[u + 4]) * inv, __uint_as_float(ov[u + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(ov[u + 6]) * inv, __uint_as_float(ov[u + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + c * 32 + u) = v;
+          for (int u2 = 0; u2 < 32; ++u2) of[u2] = __uint_as_float(ov[u2]) * inv;
+          if (valid) store_row32(orow + c * 32, of);
+        }
+        if (valid) LSE[(size_t)it.bh * N + t] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
+      } else {
+        // Split pair: every split but the last to finish leaves (O unnormalised, m, l) in its slot;
+        // the last one merges them with its own.  Counters per (pair, half): [arrivals, written].
+        int32_t* mc = fcnt + ((size_t)it.bh * n_pairs + it.kp) * 4 + h * 2;
+        if (r == 0) bar.merge_old[h] = atomicAdd(mc, 1);
+        group_sync(h);
+        const bool last = *reinterpret_cast<volatile int*>(&bar.merge_old[h]) == it.S - 1;
+        const float mo = own ? m_used : -INFINITY, lo = own ? l : 0.f;
+        if (!last) {
+          float* po = fpart + ((size_t)it.slot * 2 + h) * D * kBlockQ;
+          float* pml = fml + ((size_t)it.slot * 2 + h) * 2 * kBlockQ;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tc::tmem_ld32(tO + c * 32, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2) po[(size_t)(c * 32 + u2) * kBlockQ + r] = own ? __uint_as_float(ov[u2]) : 0.f;
+          }
+          pml[r] = mo;
+          pml[kBlockQ + r] = lo;
+          __threadfence();
+          group_sync(h);
+          if (r == 0) atomicAdd(mc + 1, 1);
+        } else {
+          if (r == 0) {   // the others have arrived: wait (bounded) until their partials are written
+            const long long c0 = clock64();
+            while (ld_acquire(mc + 1) < it.S - 1) {
+              if (clock64() - c0 > 4000000000LL) {
+                *abort_flag = 1;
+                atomicOr(status, kErrTimeoutMerge);
+                break;
+              }
+              __nanosleep(100);
             }
-          } else {
+          }
+          group_sync(h);
+          __threadfence();
+          const size_t slot0 = (size_t)(it.slot - it.s);
+          float mp[kMaxSplits], fp[kMaxSplits];
+          float M = mo;
 #pragma unroll
-            for (int u = 0; u < 32; u += 4)
-              *reinterpret_cast<float4*>(orow + c * 32 + u) =
-                  make_float4(__uint_as_float(ov[u]) * inv, __uint_as_float(ov[u + 1]) * inv,
-                              __uint_as_float(ov[u + 2]) * inv, __uint_as_float(ov[u + 3]) * inv);
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            mp[s2] = (s2 < it.S && s2 != it.s) ? __ldcg(fml + ((slot0 + s2) * 2 + h) * 2 * kBlockQ + r) : -INFINITY;
+            M = fmaxf(M, mp[s2]);
+          }
+          const float Mb = M == -INFINITY ? 0.f : M;
+          const float fo = mo == -INFINITY ? 0.f : fast_exp2(mo - Mb);
+          float L = lo * fo;
+#pragma unroll
+          for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+            fp[s2] = mp[s2] == -INFINITY ? 0.f : fast_exp2(mp[s2] - Mb);
+            if (fp[s2] != 0.f) L += __ldcg(fml + ((slot0 + s2) * 2 + h) * 2 * kBlockQ + kBlockQ + r) * fp[s2];
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tc::tmem_ld32(tO + c * 32, ov);
+            tc::tmem_wait_ld();
+            float of[32];
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2) of[u2] = fo != 0.f ? __uint_as_float(ov[u2]) * fo : 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < kMaxSplits; ++s2) {
+              if (fp[s2] == 0.f) continue;
+              const float* po = fpart + ((slot0 + s2) * 2 + h) * D * kBlockQ + (size_t)(c * 32) * kBlockQ + r;
+#pragma unroll
+              for (int u2 = 0; u2 < 32; ++u2) of[u2] = fmaf(__ldcg(po + (size_t)u2 * kBlockQ), fp[s2], of[u2]);
+            }
+#pragma unroll
+            for (int u2 = 0; u2 < 32; ++u2) of[u2] *= inv;
+            if (valid) store_row32(orow + c * 32, of);
+          }
+          if (valid) LSE[(size_t)it.bh * N + t] = (Mb + __log2f(L)) * kLn2;
+          group_sync(h);
+          if (r == 0) {   // leave the counters at zero for the next launch on the same mask
+            mc[0] = 0;
+            mc[1] = 0;
           }
         }
       }
-      if (valid) LSE[(size_t)it.bh * N + t] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
       tc::fence_before();
       tcount += n_tiles;
     }
@@ -690,16 +798,18 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
   auto k = attn_fwd_tc_kernel<D, OutT>;
   const int smem = TcSmem<D>::kBytes;
   { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
-  // persistent: one CTA per SM (the shared-memory footprint admits one), at most one per item
-  const int n_items = P.B * P.H * P.n_pairs;
-  const int grid = n_items < sm_count() ? n_items : sm_count();
+  // persistent: one CTA per SM (the shared-memory footprint admits one), at most one per unit
+  const int grid = P.sched.n_units < sm_count() ? P.sched.n_units : sm_count();
+  if (grid <= 0) return cudaSuccess;
   // delta and e enter through the per-entry metadata that the list kernel wrote beside the lists
   (void)delta;
   (void)evict;
-  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists),
-                                   ws_ptr<int32_t>(ws, P.off_pje), ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE,
-                                   ws_ptr<int32_t>(ws, P.off_status), P.B * P.H, P.H, P.G, P.N, P.n_pairs,
-                                   P.pair_cap, P.scale * kLog2e);
+  k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, P.sched, ws_ptr<int32_t>(ws, P.off_pcounts),
+                                   ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
+                                   ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE, ws_ptr<float>(ws, P.off_fpart),
+                                   ws_ptr<float>(ws, P.off_fml), ws_ptr<int32_t>(ws, P.off_fcnt),
+                                   ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_pairs, P.pair_cap,
+                                   P.scale * kLog2e);
   return cudaGetLastError();
 }
 

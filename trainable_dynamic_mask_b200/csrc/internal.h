@@ -20,6 +20,21 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Segment length of the top-w rank computation for a row of N keys: about 8 segments per row.
 inline int topw_seg_len(int N) { return N <= 4096 ? 512 : N <= 8192 ? 1024 : 2048; }
 
+// Attention-forward work schedule.  A work unit is one split of a pair of query blocks (b, h, kp):
+// pairs with long live lists are split into S parts of their list (partial results merged by the
+// unit that finishes last), so that a problem with few heavy pairs still spreads evenly over the
+// SMs.  Units are enumerated group by group (a group = one kp, its S, every (b, h)), heaviest
+// groups first; inside a group unit index = start + bh * S + s.
+constexpr int kMaxPairs = (kTopwMaxN + 2 * DMA_BLOCK_Q - 1) / (2 * DMA_BLOCK_Q);
+constexpr int kMaxSplits = 4;
+struct FwdGroup {
+  int kp, S, start, slot;   // slot: first partial-result slot of the group (-1 when S == 1)
+};
+struct FwdSchedule {
+  int n_groups, n_units, n_slots, pad;
+  FwdGroup g[kMaxPairs];
+};
+
 // Resolved problem and workspace plan.
 struct Plan {
   int B, H, Hkv, N, Nq, d, w, G;
@@ -42,8 +57,12 @@ struct Plan {
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
   size_t off_tw_keys;                  // top-w: sorted segments of composite keys [B, H, npad] u64
   // attention forward: live-key lists of query pairs of blocks (kPairQ rows), each entry with its
-  // j | e_j << 16 (i32) and delta_j * log2(e) (f32); [B, H, n_pairs, pair_cap], counts [.., 2]
-  size_t off_pcounts, off_plists, off_pje, off_pdl;
+  // e_j - j (i32) and delta_j * log2(e) (f32); [B, H, n_pairs, pair_cap], counts [.., 2]
+  size_t off_pcounts, off_plists, off_plen, off_pdl;
+  // attention forward split units: partial O [slot][half][D][128] f32, (m, l) [slot][half][2][128]
+  // f32, and per pair [arrivals, partials written] x 2 halves (i32, zeroed by the list kernel)
+  size_t off_fpart, off_fml, off_fcnt;
+  FwdSchedule sched;
   size_t off_gx;                       // gate backward: gx [B, H, N] f32
   size_t off_dA_part;                  // gate backward: [B*H][ceil(N/1024)] f32
   size_t off_dDelta_part;              // gate backward: [n_slices*B][Hkv*d][H] f32
@@ -51,6 +70,7 @@ struct Plan {
 };
 
 dma_status_t make_plan(const dma_params_t* p, Plan* plan);
+void fwd_schedule(const Plan& P, FwdSchedule* S);
 
 template <typename T> inline T* ws_ptr(void* ws, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);

@@ -349,9 +349,9 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
 // (j <= t0 and e_j >= t1: selected by every row of the range) come first, then the others, each
 // group in ascending key order.  One CTA scans the keys of a pair of blocks (kPairQ rows) once and
 // builds three lists from them: those of its two blocks (the mask encoding of the interface) and
-// that of the pair (the attention forward's work item), whose entries also carry j | e_j << 16
-// and delta_j * log2(e) and which is padded to a multiple of 128 entries with key -1 (masked for
-// every row: e = 0).
+// that of the pair (the attention forward's work item), whose entries also carry e_j - j (the
+// number of queries selecting the key) and delta_j * log2(e), and which is padded to a multiple of
+// 128 entries with key -1 and e - j = 0 (masked for every row).
 constexpr int kListThreads = 256;
 constexpr int kListWarps = kListThreads / 32;
 constexpr int kListBits = 10;                    // packed per-warp counters (a warp counts <= 128)
@@ -361,8 +361,8 @@ __global__ void __launch_bounds__(kListThreads)
 topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
                   int32_t* __restrict__ counts, int32_t* __restrict__ lists,
                   int32_t* __restrict__ pcounts, int32_t* __restrict__ plists,
-                  int32_t* __restrict__ pje, float* __restrict__ pdl, int N, int list_cap, int pair_cap,
-                  int n_blocks, int n_pairs) {
+                  int32_t* __restrict__ plen, float* __restrict__ pdl, int32_t* __restrict__ fcnt, int N,
+                  int list_cap, int pair_cap, int n_blocks, int n_pairs) {
   // partial keys: block a (<= 2C), block b (<= 2C), pair (<= 4C)
   __shared__ int32_t part[8 * kC];
   __shared__ int32_t wsum[6][kListWarps];   // per warp: full count of list 0..2, partial count of 0..2
@@ -384,9 +384,11 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
   out[1] = has_b ? out[0] + list_cap : out[0];
   const size_t pbase = ((size_t)row * n_pairs + kp) * pair_cap;
   out[2] = plists + pbase;
-  int32_t* oje = pje + pbase;
+  int32_t* olen = plen + pbase;
   float* odl = pdl + pbase;
   int nfull[3] = {0, 0, 0}, npart[3] = {0, 0, 0};
+  // the attention forward's merge counters of this pair start at zero for every new mask
+  if (tid < 4) fcnt[((size_t)row * n_pairs + kp) * 4 + tid] = 0;
   // e_j and delta_j of this thread's 4 keys, loaded one round ahead
   int enext[4];
   float dnext[4];
@@ -470,7 +472,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
           if (of[L] < cap[L]) {
             out[L][of[L]] = j;
             if (L == 2) {
-              oje[of[L]] = (j & 0xffff) | (ecur[u] << 16);
+              olen[of[L]] = ecur[u] - j;
               odl[of[L]] = dcur[u] * kLog2e;
             }
           }
@@ -503,7 +505,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
       const int j = part[poff[L] + i];
       out[L][nfull[L] + i] = j;
       if (L == 2) {
-        oje[nfull[L] + i] = (j & 0xffff) | (erow[j] << 16);
+        olen[nfull[L] + i] = erow[j] - j;
         odl[nfull[L] + i] = drow[j] * kLog2e;
       }
     }
@@ -512,7 +514,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
   const int nround = min(pair_cap, (nlive + kC - 1) / kC * kC);
   for (int i = nlive + tid; i < nround; i += kListThreads) {
     out[2][i] = -1;
-    oje[i] = 0xffff;
+    olen[i] = 0;
     odl[i] = 0.f;
   }
   if (tid == 0) {
@@ -665,8 +667,9 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
   topw_lists_kernel<<<dim3(P.n_pairs, rows), kListThreads, 0, s>>>(
       evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
-      ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_pje),
-      ws_ptr<float>(ws, P.off_pdl), P.N, P.list_cap, P.pair_cap, P.n_blocks, P.n_pairs);
+      ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
+      ws_ptr<float>(ws, P.off_pdl), ws_ptr<int32_t>(ws, P.off_fcnt), P.N, P.list_cap, P.pair_cap, P.n_blocks,
+      P.n_pairs);
   return cudaGetLastError();
 }
 
