@@ -289,14 +289,39 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
 #pragma unroll
   for (int c = 0; c < PL; ++c) acc[c] = 0.f;
   const int k0 = s * kDecodeSplit, k1 = min(sel_len, k0 + kDecodeSplit);
-  for (int kk = k0 + warp * 4 + grp; kk < k1; kk += kDecThreads / 8) {
-    const int j = srow[kk];
-    uint4 kv[PL / 8], vv[PL / 8];
+  // This lane group's keys: kk = k0 + warp * 4 + grp + it * kStride.  All their indices are loaded
+  // first, and each key's K and V rows one key ahead, so that HBM latencies overlap.
+  constexpr int kStride = kDecThreads / 8;
+  constexpr int kMaxIt = (kDecodeSplit + kStride - 1) / kStride;
+  const int kfirst = k0 + warp * 4 + grp;
+  int jl[kMaxIt];
+#pragma unroll
+  for (int it = 0; it < kMaxIt; ++it) {
+    const int kk = kfirst + it * kStride;
+    jl[it] = kk < k1 ? srow[kk] : -1;
+  }
+  uint4 kv[PL / 8], vv[PL / 8], kn[PL / 8], vn[PL / 8];
+#pragma unroll
+  for (int c = 0; c < PL / 8; ++c) kn[c] = vn[c] = make_uint4(0, 0, 0, 0);
+  auto load_rows = [&](int j, uint4 (&kr)[PL / 8], uint4 (&vr)[PL / 8]) {
 #pragma unroll
     for (int c = 0; c < PL / 8; ++c) {
-      kv[c] = *reinterpret_cast<const uint4*>(Kg + (size_t)j * D + sub * PL + c * 8);
-      vv[c] = *reinterpret_cast<const uint4*>(Vg + (size_t)j * D + sub * PL + c * 8);
+      kr[c] = *reinterpret_cast<const uint4*>(Kg + (size_t)j * D + sub * PL + c * 8);
+      vr[c] = *reinterpret_cast<const uint4*>(Vg + (size_t)j * D + sub * PL + c * 8);
     }
+  };
+  if (jl[0] >= 0) load_rows(jl[0], kn, vn);
+#pragma unroll
+  for (int it = 0; it < kMaxIt; ++it) {
+    const int j = jl[it];
+    // the shuffles below involve the whole warp: stop only when no lane group has a key left
+    if (!__any_sync(0xffffffffu, j >= 0)) break;
+#pragma unroll
+    for (int c = 0; c < PL / 8; ++c) {
+      kv[c] = kn[c];
+      vv[c] = vn[c];
+    }
+    if (it + 1 < kMaxIt && jl[it + 1] >= 0) load_rows(jl[it + 1], kn, vn);
     float dot = 0.f;
 #pragma unroll
     for (int c = 0; c < PL / 8; ++c) {
@@ -310,6 +335,7 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
     dot += __shfl_xor_sync(0xffffffffu, dot, 1);
     dot += __shfl_xor_sync(0xffffffffu, dot, 2);
     dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+    if (j < 0) continue;   // this group's keys are done (its registers hold no loaded rows)
     const float x = fmaf(dot, scale_log2, drow[j] * kLog2e);
     const float mn = fmaxf(m, x);
     const float a = fast_exp2(m - mn), p = fast_exp2(x - mn);

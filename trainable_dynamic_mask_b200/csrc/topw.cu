@@ -534,14 +534,67 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
 // ---------------------------------------------------------------- decode selection
 
 constexpr int kSelThreads = 1024;
+constexpr int kSelBatch = 8;                   // rounds of loads issued together
+constexpr int kSelBits = 12;                   // histogram window
+constexpr int kSelBins = 1 << kSelBits;
+constexpr int kSelCand = 6144;                 // candidates kept in shared memory
+constexpr int kSelWarps = kSelThreads / 32;
 
-// Top-w of the whole row (query at position N-1): 4-pass MSB-first radix select on the order key,
-// then an order-preserving compaction of the selected positions.
-__global__ void __launch_bounds__(kSelThreads)
+struct SelShared {
+  uint32_t hist[kSelBins];
+  uint32_t cand_key[kSelCand];
+  uint32_t red[2][kSelWarps];
+  int32_t scan[2][kSelBatch * kSelWarps];   // exclusive prefix of (greater, equal) counts per (round, warp)
+  uint32_t bin, above, ncand;
+};
+
+// The bin (from the highest) in which the count accumulated from the highest bin reaches `need`,
+// and the count of the bins above it, into S.bin / S.above.  hist must be complete.
+DMA_DEVINL void sel_find_bin(SelShared& S, uint32_t need, int nbins, int tid) {
+  if (tid < 32) {
+    const int lane = tid;
+    const int per = (nbins + 31) / 32;   // bins per lane, lane 0 takes the highest
+    uint32_t sum = 0;
+    for (int u = 0; u < per; ++u) {
+      const int q = lane * per + u;
+      if (q < nbins) sum += S.hist[nbins - 1 - q];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need);
+    const int l = __ffs(hit) - 1;
+    if (lane == l) {
+      uint32_t above = incl - sum;
+      for (int u = 0; u < per; ++u) {
+        const int q = lane * per + u;
+        if (q >= nbins) break;
+        const uint32_t bin = (uint32_t)(nbins - 1 - q);
+        if (above + S.hist[bin] >= need) {
+          S.bin = bin;
+          S.above = above;
+          break;
+        }
+        above += S.hist[bin];
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Top-w of the whole row (the query at position N-1), in the order (delta desc, index asc).
+// Selection by histograms over a 12-bit window of the order key, starting at the highest bit in
+// which the row's keys differ (delta values crowd into a few exponents, so a fixed top-byte pass
+// would separate almost nothing).  Passes over the row narrow the window until the bin holding the
+// w-th best key has at most kSelCand keys; those are then resolved in shared memory.  A last pass
+// writes the selected positions in ascending order.
+__global__ void __launch_bounds__(kSelThreads, 1)
 topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int N, int w) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t sh_prefix, sh_need;
-  __shared__ int32_t wcnt[2][kSelThreads / 32];
+  extern __shared__ __align__(16) unsigned char sel_raw[];
+  SelShared& S = *reinterpret_cast<SelShared*>(sel_raw);
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* drow = delta + (size_t)row * N;
@@ -551,82 +604,165 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
     for (int i = tid; i < N; i += kSelThreads) out[i] = i;
     return;
   }
-  uint32_t prefix = 0, mask = 0, need = (uint32_t)k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int i0 = 0; i0 < N; i0 += kSelThreads) {
-      const int i = i0 + tid;
-      const bool valid = i < N;
-      uint32_t key = valid ? order_key(drow[i]) : 0u;
-      const bool in = valid && ((key & mask) == prefix);
-      const uint32_t imask = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const uint32_t dig = (key >> shift) & 255u;
-        const uint32_t peers = __match_any_sync(imask, dig);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[dig], __popc(peers));
+  // ---- key range of the row
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int i0 = 0; i0 < N; i0 += kSelThreads * kSelBatch) {
+    uint32_t kb[kSelBatch];
+#pragma unroll
+    for (int u = 0; u < kSelBatch; ++u) {
+      const int i = i0 + u * kSelThreads + tid;
+      kb[u] = i < N ? order_key(drow[i]) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kSelBatch; ++u) {
+      if (i0 + u * kSelThreads + tid < N) {
+        kmin = min(kmin, kb[u]);
+        kmax = max(kmax, kb[u]);
       }
     }
-    __syncthreads();
-    if (warp == 0) {
-      // digits from high to low: lane l owns digits 255-8l .. 248-8l
-      uint32_t v[8], s = 0;
+  }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) { v[u] = hist[255 - (lane * 8 + u)]; s += v[u]; }
-      uint32_t incl = s;
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) { S.red[0][warp] = kmin; S.red[1][warp] = kmax; }
+  __syncthreads();
+  kmin = 0xffffffffu;
+  kmax = 0u;
+  for (int i = 0; i < kSelWarps; ++i) { kmin = min(kmin, S.red[0][i]); kmax = max(kmax, S.red[1][i]); }
+  __syncthreads();
+  // ---- narrowing.  Keys in play: (key >> (shift + width)) == pre, where [shift, shift + width) is
+  // the current window; when every key is equal the threshold is that key.
+  uint32_t need = (uint32_t)k;
+  uint32_t thr = kmin;
+  if (kmin != kmax) {
+    const int top = 31 - __clz(kmin ^ kmax);   // highest bit in which the keys differ
+    int width = top + 1 < kSelBits ? top + 1 : kSelBits;
+    int shift = top + 1 - width;
+    uint32_t pre = top == 31 ? 0u : kmin >> (top + 1);
+    bool in_smem = false;   // candidates collected in shared memory
+    int ncand = 0;
+    while (true) {
+      // histogram of the window over the keys in play
+      for (int i = tid; i < kSelBins; i += kSelThreads) S.hist[i] = 0;
+      __syncthreads();
+      const uint32_t wmask = (1u << width) - 1u;
+      const int hs = shift + width;   // bits above the window
+      if (!in_smem) {
+        for (int i0 = 0; i0 < N; i0 += kSelThreads * kSelBatch) {
+          uint32_t kb[kSelBatch];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t hit = __ballot_sync(0xffffffffu, incl >= need);
-      const int l = __ffs(hit) - 1;
-      if (lane == l) {
-        uint32_t above = incl - s;
-        for (int u = 0; u < 8; ++u) {
-          if (above + v[u] >= need) {
-            sh_prefix = prefix | ((uint32_t)(255 - (lane * 8 + u)) << shift);
-            sh_need = need - above;
-            break;
+          for (int u = 0; u < kSelBatch; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            kb[u] = i < N ? order_key(drow[i]) : 0u;
           }
-          above += v[u];
+#pragma unroll
+          for (int u = 0; u < kSelBatch; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            const uint32_t hi = hs >= 32 ? 0u : kb[u] >> hs;
+            if (i < N && hi == pre) atomicAdd(&S.hist[(kb[u] >> shift) & wmask], 1u);
+          }
+        }
+      } else {
+        for (int c = tid; c < ncand; c += kSelThreads) {
+          const uint32_t key = S.cand_key[c];
+          const uint32_t hi = hs >= 32 ? 0u : key >> hs;
+          if (hi == pre) atomicAdd(&S.hist[(key >> shift) & wmask], 1u);
         }
       }
+      __syncthreads();
+      sel_find_bin(S, need, 1 << width, tid);
+      const uint32_t bin = S.bin, cnt = S.hist[S.bin];
+      need -= S.above;
+      pre = (hs >= 32 ? 0u : pre << width) | bin;
+      __syncthreads();
+      if (shift == 0) {   // the bin is a single key value
+        thr = pre;
+        break;
+      }
+      if (!in_smem && cnt <= (uint32_t)kSelCand) {
+        // collect the bin's keys (their order does not matter: only the threshold is sought)
+        if (tid == 0) S.ncand = 0;
+        __syncthreads();
+        for (int i0 = 0; i0 < N; i0 += kSelThreads * kSelBatch) {
+          uint32_t kb[kSelBatch];
+#pragma unroll
+          for (int u = 0; u < kSelBatch; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            kb[u] = i < N ? order_key(drow[i]) : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < kSelBatch; ++u) {
+            const int i = i0 + u * kSelThreads + tid;
+            if (i < N && (kb[u] >> shift) == pre) {
+              const uint32_t slot = atomicAdd(&S.ncand, 1u);
+              if (slot < (uint32_t)kSelCand) S.cand_key[slot] = kb[u];
+            }
+          }
+        }
+        __syncthreads();
+        ncand = (int)min(S.ncand, (uint32_t)kSelCand);
+        in_smem = true;
+      }
+      width = shift < kSelBits ? shift : kSelBits;
+      shift -= width;
+      __syncthreads();
     }
-    __syncthreads();
-    prefix = sh_prefix;
-    need = sh_need;
-    mask |= 255u << shift;
-    __syncthreads();
   }
-  // prefix = order key of the k-th best; take keys above it and the first `need` equal ones
-  int taken = 0, eqseen = 0;
-  for (int i0 = 0; i0 < N; i0 += kSelThreads) {
-    const int i = i0 + tid;
-    const uint32_t key = i < N ? order_key(drow[i]) : 0u;
-    const bool gt = i < N && key > prefix;
-    const bool eq = i < N && key == prefix;
-    const uint32_t meq = __ballot_sync(0xffffffffu, eq);
-    int eq_before_in_warp = __popc(meq & lanemask_lt());
-    if (lane == 0) wcnt[1][warp] = __popc(meq);
-    __syncthreads();
-    int eq_before = eqseen + eq_before_in_warp, eq_tot = 0;
-    for (int u = 0; u < kSelThreads / 32; ++u) {
-      if (u < warp) eq_before += wcnt[1][u];
-      eq_tot += wcnt[1][u];
+  // ---- thr = key of the k-th best: take keys above it and the first `need` equal ones, in index
+  // order.  out position of a taken key = #greater before it + min(#equal before it, need).
+  int gt_run = 0, eq_run = 0;
+  for (int i0 = 0; i0 < N; i0 += kSelThreads * kSelBatch) {
+    uint32_t kb[kSelBatch];
+#pragma unroll
+    for (int u = 0; u < kSelBatch; ++u) {
+      const int i = i0 + u * kSelThreads + tid;
+      kb[u] = i < N ? order_key(drow[i]) : 0u;
     }
-    const bool take = gt || (eq && eq_before < (int)need);
-    const uint32_t mt = __ballot_sync(0xffffffffu, take);
-    if (lane == 0) wcnt[0][warp] = __popc(mt);
-    __syncthreads();
-    int t_before = taken + __popc(mt & lanemask_lt()), t_tot = 0;
-    for (int u = 0; u < kSelThreads / 32; ++u) {
-      if (u < warp) t_before += wcnt[0][u];
-      t_tot += wcnt[0][u];
+    uint32_t mg[kSelBatch], me[kSelBatch];
+#pragma unroll
+    for (int u = 0; u < kSelBatch; ++u) {
+      const bool in = i0 + u * kSelThreads + tid < N;
+      mg[u] = __ballot_sync(0xffffffffu, in && kb[u] > thr);
+      me[u] = __ballot_sync(0xffffffffu, in && kb[u] == thr);
+      if (lane == 0) {
+        S.scan[0][u * kSelWarps + warp] = __popc(mg[u]);
+        S.scan[1][u * kSelWarps + warp] = __popc(me[u]);
+      }
     }
-    if (take && t_before < k) out[t_before] = i;
-    taken += t_tot;
-    eqseen += eq_tot;
+    __syncthreads();
+    if (warp < 2) {   // exclusive scans in (round, warp) order: warp 0 the greater, warp 1 the equal
+      constexpr int kPer = kSelBatch * kSelWarps / 32;
+      int v[kPer], sum = 0;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) { v[u] = S.scan[warp][lane * kPer + u]; sum += v[u]; }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - sum;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) { S.scan[warp][lane * kPer + u] = run; run += v[u]; }
+      if (lane == 31) S.red[warp][0] = (uint32_t)run;   // batch totals
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kSelBatch; ++u) {
+      const int i = i0 + u * kSelThreads + tid;
+      const uint32_t lt = (1u << lane) - 1u;
+      const int gb = gt_run + S.scan[0][u * kSelWarps + warp] + __popc(mg[u] & lt);
+      const int eb = eq_run + S.scan[1][u * kSelWarps + warp] + __popc(me[u] & lt);
+      const bool g = (mg[u] >> lane) & 1u, e = (me[u] >> lane) & 1u;
+      if (g || (e && eb < (int)need)) {
+        const int o = gb + min(eb, (int)need);
+        if (o < k) out[o] = i;
+      }
+    }
+    gt_run += (int)S.red[0][0];
+    eq_run += (int)S.red[1][0];
     __syncthreads();
   }
 }
@@ -674,8 +810,9 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
 }
 
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
-  topw_decode_kernel<<<P.B * P.H, kSelThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N,
-                                                       P.w);
+  const int smem = (int)sizeof(SelShared);
+  { cudaError_t ea = ensure_smem_limit(topw_decode_kernel, smem); if (ea != cudaSuccess) return ea; }
+  topw_decode_kernel<<<P.B * P.H, kSelThreads, smem, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w);
   return cudaGetLastError();
 }
 
