@@ -290,9 +290,12 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
   for (int c = 0; c < PL; ++c) acc[c] = 0.f;
   const int k0 = s * kDecodeSplit, k1 = min(sel_len, k0 + kDecodeSplit);
   // This lane group's keys: kk = k0 + warp * 4 + grp + it * kStride.  All their indices are loaded
-  // first, and each key's K and V rows one key ahead, so that HBM latencies overlap.
+  // first; then the K and V rows of kChunk keys at a time are loaded together before any is used,
+  // so that each lane keeps 4 KB of row loads of its warp in flight.
   constexpr int kStride = kDecThreads / 8;
   constexpr int kMaxIt = (kDecodeSplit + kStride - 1) / kStride;
+  constexpr int kChunk = 4;
+  static_assert(kMaxIt % kChunk == 0, "chunks of keys per lane group");
   const int kfirst = k0 + warp * 4 + grp;
   int jl[kMaxIt];
 #pragma unroll
@@ -300,54 +303,51 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
     const int kk = kfirst + it * kStride;
     jl[it] = kk < k1 ? srow[kk] : -1;
   }
-  uint4 kv[PL / 8], vv[PL / 8], kn[PL / 8], vn[PL / 8];
 #pragma unroll
-  for (int c = 0; c < PL / 8; ++c) kn[c] = vn[c] = make_uint4(0, 0, 0, 0);
-  auto load_rows = [&](int j, uint4 (&kr)[PL / 8], uint4 (&vr)[PL / 8]) {
-#pragma unroll
-    for (int c = 0; c < PL / 8; ++c) {
-      kr[c] = *reinterpret_cast<const uint4*>(Kg + (size_t)j * D + sub * PL + c * 8);
-      vr[c] = *reinterpret_cast<const uint4*>(Vg + (size_t)j * D + sub * PL + c * 8);
-    }
-  };
-  if (jl[0] >= 0) load_rows(jl[0], kn, vn);
-#pragma unroll
-  for (int it = 0; it < kMaxIt; ++it) {
-    const int j = jl[it];
+  for (int it0 = 0; it0 < kMaxIt; it0 += kChunk) {
     // the shuffles below involve the whole warp: stop only when no lane group has a key left
-    if (!__any_sync(0xffffffffu, j >= 0)) break;
+    if (!__any_sync(0xffffffffu, jl[it0] >= 0)) break;
+    uint4 kr[kChunk][PL / 8], vr[kChunk][PL / 8];
+    float dl[kChunk];
 #pragma unroll
-    for (int c = 0; c < PL / 8; ++c) {
-      kv[c] = kn[c];
-      vv[c] = vn[c];
-    }
-    if (it + 1 < kMaxIt && jl[it + 1] >= 0) load_rows(jl[it + 1], kn, vn);
-    float dot = 0.f;
+    for (int c4 = 0; c4 < kChunk; ++c4) {
+      const int j = jl[it0 + c4];
 #pragma unroll
-    for (int c = 0; c < PL / 8; ++c) {
-      const uint32_t w4[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        dot = fmaf(q[c * 8 + 2 * u], __uint_as_float(w4[u] << 16), dot);
-        dot = fmaf(q[c * 8 + 2 * u + 1], __uint_as_float(w4[u] & 0xffff0000u), dot);
+      for (int c = 0; c < PL / 8; ++c) {
+        kr[c4][c] = j >= 0 ? *reinterpret_cast<const uint4*>(Kg + (size_t)j * D + sub * PL + c * 8) : make_uint4(0, 0, 0, 0);
+        vr[c4][c] = j >= 0 ? *reinterpret_cast<const uint4*>(Vg + (size_t)j * D + sub * PL + c * 8) : make_uint4(0, 0, 0, 0);
       }
+      dl[c4] = j >= 0 ? drow[j] * kLog2e : 0.f;
     }
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 4);
-    if (j < 0) continue;   // this group's keys are done (its registers hold no loaded rows)
-    const float x = fmaf(dot, scale_log2, drow[j] * kLog2e);
-    const float mn = fmaxf(m, x);
-    const float a = fast_exp2(m - mn), p = fast_exp2(x - mn);
-    m = mn;
-    l = l * a + p;
 #pragma unroll
-    for (int c = 0; c < PL / 8; ++c) {
-      const uint32_t w4[4] = {vv[c].x, vv[c].y, vv[c].z, vv[c].w};
+    for (int c4 = 0; c4 < kChunk; ++c4) {
+      float dot = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc[c * 8 + 2 * u] = fmaf(p, __uint_as_float(w4[u] << 16), acc[c * 8 + 2 * u] * a);
-        acc[c * 8 + 2 * u + 1] = fmaf(p, __uint_as_float(w4[u] & 0xffff0000u), acc[c * 8 + 2 * u + 1] * a);
+      for (int c = 0; c < PL / 8; ++c) {
+        const uint32_t w4[4] = {kr[c4][c].x, kr[c4][c].y, kr[c4][c].z, kr[c4][c].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          dot = fmaf(q[c * 8 + 2 * u], __uint_as_float(w4[u] << 16), dot);
+          dot = fmaf(q[c * 8 + 2 * u + 1], __uint_as_float(w4[u] & 0xffff0000u), dot);
+        }
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 4);
+      if (jl[it0 + c4] < 0) continue;
+      const float x = fmaf(dot, scale_log2, dl[c4]);
+      const float mn = fmaxf(m, x);
+      const float a = fast_exp2(m - mn), p = fast_exp2(x - mn);
+      m = mn;
+      l = l * a + p;
+#pragma unroll
+      for (int c = 0; c < PL / 8; ++c) {
+        const uint32_t w4[4] = {vr[c4][c].x, vr[c4][c].y, vr[c4][c].z, vr[c4][c].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          acc[c * 8 + 2 * u] = fmaf(p, __uint_as_float(w4[u] << 16), acc[c * 8 + 2 * u] * a);
+          acc[c * 8 + 2 * u + 1] = fmaf(p, __uint_as_float(w4[u] & 0xffff0000u), acc[c * 8 + 2 * u + 1] * a);
+        }
       }
     }
   }

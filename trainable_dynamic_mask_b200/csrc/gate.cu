@@ -187,71 +187,118 @@ __global__ void gate_bwd_pointwise_kernel(const float* __restrict__ x, const flo
 }
 
 // dV_gate[b,g,j,c] = sum_h gx[b,h,j] * Delta[g*d+c, h]
-template <typename T>
-__global__ void gate_bwd_dv_kernel(const float* __restrict__ gx, const T* __restrict__ Delta,
-                                   float* __restrict__ dVg, int H, int Hkv, int N, int d) {
-  extern __shared__ float sm[];
-  float* Gs = sm;                 // [H][kGatePT]
-  float* Ds = sm + H * kGatePT;   // [d][H]
-  const int b = blockIdx.y, j0 = blockIdx.x * kGatePT;
-  for (int e = threadIdx.x; e < H * kGatePT; e += blockDim.x) {
-    int h = e / kGatePT, p = e % kGatePT;
+// dV_gate[b, g, j, c] = sum_h gx[b, h, j] Delta[g d + c, h]: per (64 positions, g, b) a
+// [64 x H] x [H x d] product in float32.  Thread = PP = d / 32 positions x 8 channels (register
+// tile), reading gx as [h][64 positions] and Delta as [h][d] from shared memory with 16-byte loads;
+// a warp stores 512 contiguous bytes per position.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+gate_bwd_dv_kernel(const float* __restrict__ gx, const T* __restrict__ Delta, float* __restrict__ dVg, int H,
+                   int Hkv, int N) {
+  constexpr int CG = D / 8, PP = kGatePT * CG / 256;   // channel groups; positions per thread
+  extern __shared__ __align__(16) float sm[];
+  float* Gs = sm;                    // [H][kGatePT]
+  float* Ds = sm + H * kGatePT;      // [H][D]
+  const int j0 = blockIdx.x * kGatePT, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, cg = tid % CG, pg = tid / CG;
+  for (int e = tid; e < H * kGatePT; e += 256) {
+    const int h = e / kGatePT, p = e % kGatePT;
     Gs[e] = (j0 + p < N) ? gx[(size_t)(b * H + h) * N + j0 + p] : 0.f;
   }
-  for (int g = 0; g < Hkv; ++g) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < d * H; e += blockDim.x) Ds[e] = load_as_f32(Delta + (size_t)g * d * H + e);
-    __syncthreads();
-    for (int e = threadIdx.x; e < kGatePT * d; e += blockDim.x) {
-      const int p = e / d, c = e % d;
-      if (j0 + p >= N) continue;
-      float acc = 0.f;
-      for (int h = 0; h < H; ++h) acc = fmaf(Gs[h * kGatePT + p], Ds[c * H + h], acc);
-      dVg[((size_t)(b * Hkv + g) * N + j0 + p) * d + c] = acc;
-    }
+  for (int e = tid; e < D * H; e += 256) {
+    const int c = e / H, h = e % H;   // coalesced over the row-major Delta
+    Ds[h * D + c] = load_as_f32(Delta + (size_t)(g * D + c) * H + h);
+  }
+  __syncthreads();
+  float acc[PP][8];
+#pragma unroll
+  for (int p = 0; p < PP; ++p)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[p][c] = 0.f;
+  for (int h = 0; h < H; ++h) {
+    const float4 d0 = *reinterpret_cast<const float4*>(Ds + h * D + cg * 8);
+    const float4 d1 = *reinterpret_cast<const float4*>(Ds + h * D + cg * 8 + 4);
+    const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+    float gg[PP];
+#pragma unroll
+    for (int p = 0; p < PP; ++p) gg[p] = Gs[h * kGatePT + pg * PP + p];
+#pragma unroll
+    for (int p = 0; p < PP; ++p)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[p][c] = fmaf(gg[p], dd[c], acc[p][c]);
+  }
+#pragma unroll
+  for (int p = 0; p < PP; ++p) {
+    const int j = j0 + pg * PP + p;
+    if (j >= N) continue;
+    float* o = dVg + ((size_t)(b * Hkv + g) * N + j) * D + cg * 8;
+    *reinterpret_cast<float4*>(o) = make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
+    *reinterpret_cast<float4*>(o + 4) = make_float4(acc[p][4], acc[p][5], acc[p][6], acc[p][7]);
   }
 }
 
-// partial[(s*B + b)][g*d + c][h] = sum_{j in slice s} V[b,g,j,c] * gx[b,h,j]
-template <typename T>
-__global__ void gate_bwd_ddelta_partial_kernel(const T* __restrict__ V, const float* __restrict__ gx,
-                                               float* __restrict__ part, int B, int H, int Hkv,
-                                               int N, int d) {
-  extern __shared__ float sm[];
-  float* Vs = sm;                   // [64][d]
-  float* Gs = sm + 64 * d;          // [H][64]
+// partial[(s*B + b)][g*d + c][h] = sum_{j in slice s} V[b,g,j,c] * gx[b,h,j].  Thread = 8 channels x
+// 4 heads (register tile); the NT = (d / 8) x ceil(H / 4) tiles are repeated 256 / NT times over
+// disjoint positions of each 64-position chunk and summed through shared memory at the end.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+gate_bwd_ddelta_partial_kernel(const T* __restrict__ V, const float* __restrict__ gx, float* __restrict__ part,
+                               int B, int H, int Hkv, int N) {
+  constexpr int CG = D / 8;
+  extern __shared__ __align__(16) float sm[];
+  const int HG = (H + 3) / 4, HP = HG * 4, NT = CG * HG, NQ = 256 / NT;
+  float* Vs = sm;                    // [64][D]
+  float* Gs = sm + 64 * D;           // [64][HP]
+  float* red = Gs + 64 * HP;         // [NQ][NT][32]
   const int s = blockIdx.x, b = blockIdx.y, g = blockIdx.z;
-  const int c = threadIdx.x % d;
-  const int hg = threadIdx.x / d, nhg = blockDim.x / d;
-  float acc[32];
+  const int tid = threadIdx.x;
+  const int q = tid / NT, t = tid % NT, cg = t % CG, hg = t / CG;
+  float acc[8][4];
 #pragma unroll
-  for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-  const T* Vg = V + (size_t)(b * Hkv + g) * N * d;
-  for (int j0 = s * kGateSlice; j0 < min(N, (s + 1) * kGateSlice); j0 += 64) {
+  for (int c = 0; c < 8; ++c)
+#pragma unroll
+    for (int h = 0; h < 4; ++h) acc[c][h] = 0.f;
+  const T* Vg = V + (size_t)(b * Hkv + g) * N * D;
+  const int jend = min(N, (s + 1) * kGateSlice);
+  for (int j0 = s * kGateSlice; j0 < jend; j0 += 64) {
     __syncthreads();
-    for (int e = threadIdx.x; e < 64 * d; e += blockDim.x) {
-      const int p = e / d, cc = e % d;
-      Vs[e] = (j0 + p < N) ? load_as_f32(Vg + (size_t)(j0 + p) * d + cc) : 0.f;
+    for (int e = tid; e < 64 * D; e += 256) {
+      const int p = e / D, c = e % D;
+      Vs[e] = (j0 + p < N) ? load_as_f32(Vg + (size_t)(j0 + p) * D + c) : 0.f;
     }
-    for (int e = threadIdx.x; e < H * 64; e += blockDim.x) {
+    for (int e = tid; e < HP * 64; e += 256) {
       const int h = e / 64, p = e % 64;
-      Gs[e] = (j0 + p < N) ? gx[(size_t)(b * H + h) * N + j0 + p] : 0.f;
+      Gs[p * HP + h] = (h < H && j0 + p < N) ? gx[(size_t)(b * H + h) * N + j0 + p] : 0.f;
     }
     __syncthreads();
-    for (int p = 0; p < 64; ++p) {
-      const float v = Vs[p * d + c];
+    if (q < NQ) {
+      for (int p = q; p < 64; p += NQ) {
+        const float4 v0 = *reinterpret_cast<const float4*>(Vs + p * D + cg * 8);
+        const float4 v1 = *reinterpret_cast<const float4*>(Vs + p * D + cg * 8 + 4);
+        const float4 g4 = *reinterpret_cast<const float4*>(Gs + p * HP + hg * 4);
+        const float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const float gg[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const int h = hg + k * nhg;
-        if (h < H) acc[k] = fmaf(v, Gs[h * 64 + p], acc[k]);
+        for (int c = 0; c < 8; ++c)
+#pragma unroll
+          for (int h = 0; h < 4; ++h) acc[c][h] = fmaf(vv[c], gg[h], acc[c][h]);
       }
     }
   }
-  float* out = part + ((size_t)(s * B + b) * Hkv * d + (size_t)g * d + c) * H;
+  __syncthreads();
+  if (q < NQ) {
 #pragma unroll
-  for (int k = 0; k < 32; ++k) {
-    const int h = hg + k * nhg;
-    if (h < H) out[h] = acc[k];
+    for (int c = 0; c < 8; ++c)
+#pragma unroll
+      for (int h = 0; h < 4; ++h) red[((size_t)q * NT + t) * 32 + c * 4 + h] = acc[c][h];
+  }
+  __syncthreads();
+  for (int e = tid; e < NT * 32; e += 256) {
+    const int tt = e / 32, ch = e % 32, c = ch / 4, h = ch % 4;
+    float v = 0.f;
+    for (int qq = 0; qq < NQ; ++qq) v += red[((size_t)qq * NT + tt) * 32 + ch];
+    const int cc = (tt % CG) * 8 + c, hh = (tt / CG) * 4 + h;
+    if (hh < H) part[((size_t)(s * B + b) * Hkv * D + (size_t)g * D + cc) * H + hh] = v;
   }
 }
 
@@ -454,7 +501,7 @@ cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n
 cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             const float* x_save, const float* delta, const float* d_delta,
                             float* dDelta, float* dA, float* dV_gate, void* ws, cudaStream_t s) {
-  if (P.H > 32 * (256 / P.d)) return cudaErrorInvalidValue;
+  if ((P.d / 8) * ((P.H + 3) / 4) > 256) return cudaErrorInvalidValue;   // one register tile per thread
   float* gx = ws_ptr<float>(ws, P.off_gx);
   float* dA_part = ws_ptr<float>(ws, P.off_dA_part);
   float* part = ws_ptr<float>(ws, P.off_dDelta_part);
@@ -462,24 +509,30 @@ cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, con
   gate_bwd_pointwise_kernel<<<dim3(nchunk, P.B * P.H), 256, 0, s>>>(x_save, delta, d_delta, A, gx,
                                                                      dA_part, P.H, P.N);
   const size_t smem_dv = (size_t)(P.H * kGatePT + P.d * P.H) * sizeof(float);
-  const size_t smem_dd = (size_t)(64 * P.d + P.H * 64) * sizeof(float);
-  dim3 gdv((P.N + kGatePT - 1) / kGatePT, P.B);
+  const int HP = (P.H + 3) / 4 * 4, NT = (P.d / 8) * (HP / 4);
+  const size_t smem_dd = (size_t)(64 * P.d + 64 * HP + (256 / NT) * NT * 32) * sizeof(float);
+  dim3 gdv((P.N + kGatePT - 1) / kGatePT, P.Hkv, P.B);
   dim3 gdd(P.n_slices, P.B, P.Hkv);
+  auto launch = [&](auto kdv, auto kdd, const auto* Vp, const auto* Dp) -> cudaError_t {
+    { cudaError_t ea = ensure_smem_limit(kdv, (int)smem_dv); if (ea != cudaSuccess) return ea; }
+    kdv<<<gdv, 256, smem_dv, s>>>(gx, Dp, dV_gate, P.H, P.Hkv, P.N);
+    { cudaError_t ea = ensure_smem_limit(kdd, (int)smem_dd); if (ea != cudaSuccess) return ea; }
+    kdd<<<gdd, 256, smem_dd, s>>>(Vp, gx, part, P.B, P.H, P.Hkv, P.N);
+    return cudaSuccess;
+  };
+  cudaError_t e;
   if (P.bf16) {
-    auto k1 = gate_bwd_dv_kernel<uint16_t>;
-    { cudaError_t ea = ensure_smem_limit(k1, (int)smem_dv); if (ea != cudaSuccess) return ea; }
-    k1<<<gdv, 256, smem_dv, s>>>(gx, (const uint16_t*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
-    auto k2 = gate_bwd_ddelta_partial_kernel<uint16_t>;
-    { cudaError_t ea = ensure_smem_limit(k2, (int)smem_dd); if (ea != cudaSuccess) return ea; }
-    k2<<<gdd, 256, smem_dd, s>>>((const uint16_t*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
+    const uint16_t* Vp = (const uint16_t*)V;
+    const uint16_t* Dp = (const uint16_t*)Delta;
+    e = P.d == 128 ? launch(gate_bwd_dv_kernel<uint16_t, 128>, gate_bwd_ddelta_partial_kernel<uint16_t, 128>, Vp, Dp)
+                   : launch(gate_bwd_dv_kernel<uint16_t, 64>, gate_bwd_ddelta_partial_kernel<uint16_t, 64>, Vp, Dp);
   } else {
-    auto k1 = gate_bwd_dv_kernel<float>;
-    { cudaError_t ea = ensure_smem_limit(k1, (int)smem_dv); if (ea != cudaSuccess) return ea; }
-    k1<<<gdv, 256, smem_dv, s>>>(gx, (const float*)Delta, dV_gate, P.H, P.Hkv, P.N, P.d);
-    auto k2 = gate_bwd_ddelta_partial_kernel<float>;
-    { cudaError_t ea = ensure_smem_limit(k2, (int)smem_dd); if (ea != cudaSuccess) return ea; }
-    k2<<<gdd, 256, smem_dd, s>>>((const float*)V, gx, part, P.B, P.H, P.Hkv, P.N, P.d);
+    const float* Vp = (const float*)V;
+    const float* Dp = (const float*)Delta;
+    e = P.d == 128 ? launch(gate_bwd_dv_kernel<float, 128>, gate_bwd_ddelta_partial_kernel<float, 128>, Vp, Dp)
+                   : launch(gate_bwd_dv_kernel<float, 64>, gate_bwd_ddelta_partial_kernel<float, 64>, Vp, Dp);
   }
+  if (e != cudaSuccess) return e;
   const int RH = P.Hkv * P.d * P.H;
   gate_bwd_reduce_kernel<<<(RH + 255) / 256, 256, 0, s>>>(part, dA_part, dDelta, dA,
                                                           P.n_slices * P.B, RH, P.H, P.B, nchunk);
