@@ -155,6 +155,7 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_fml = take((size_t)R.sched.n_slots * 2 * 2 * kBlockQ * sizeof(float));
     R.off_fcnt = take(BH * R.n_pairs * 4 * sizeof(int32_t));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
+    R.off_bwd_perm = take((size_t)R.B * R.Hkv * R.N * sizeof(int32_t));
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));
     R.off_tw_T = take(BH * (R.n_blocks + 1) * sizeof(int32_t));

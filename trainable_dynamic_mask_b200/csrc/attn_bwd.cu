@@ -272,28 +272,32 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 bwd_dkv_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                const uint16_t* __restrict__ V, const uint16_t* __restrict__ dO,
                const float* __restrict__ delta, const int32_t* __restrict__ evict,
-               const float* __restrict__ LSE, const float* __restrict__ Drow, OutT* __restrict__ dK,
-               OutT* __restrict__ dV, float* __restrict__ d_delta, int H, int G, int N,
-               float scale_log2, float scale) {
+               const int32_t* __restrict__ perm, const float* __restrict__ LSE,
+               const float* __restrict__ Drow, OutT* __restrict__ dK, OutT* __restrict__ dV,
+               float* __restrict__ d_delta, int H, int G, int N, float scale_log2, float scale) {
   using S = DkvSmem<D>;
   extern __shared__ __align__(128) unsigned char sm[];
-  __shared__ int qmax_sh;
+  __shared__ int qmax_sh, qmin_sh;
+  __shared__ int tile_j[64];
   const int n_kt = (N + 63) / 64;
   const int kt = n_kt - 1 - (int)blockIdx.x;
   const int bg = blockIdx.y;   // b * Hkv + g
   const int Hkv = H / G;
   const int b = bg / Hkv, g = bg % Hkv;
-  const int j0 = kt * 64;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint16_t* Kg = K + (size_t)bg * N * D;
   const uint16_t* Vg = V + (size_t)bg * N * D;
+  // this tile's keys: entries [64 kt, 64 kt + 64) of the group's key order (N past the end)
+  if (tid < 64) tile_j[tid] = 64 * kt + tid < N ? perm[(size_t)bg * N + 64 * kt + tid] : N;
+  __syncthreads();
   {
     const uint32_t kb = smem_u32(sm), vb = smem_u32(sm + S::kOffV);
     for (int i = tid; i < 64 * S::kRowChunks; i += kDkvThreads) {
       const int r = i / S::kRowChunks, c = i % S::kRowChunks;
-      const bool ok = j0 + r < N;
-      cp_async_16(kb + swz(r, c, S::kRowChunks), Kg + (size_t)(ok ? j0 + r : 0) * D + c * 8, ok ? 16 : 0);
-      cp_async_16(vb + swz(r, c, S::kRowChunks), Vg + (size_t)(ok ? j0 + r : 0) * D + c * 8, ok ? 16 : 0);
+      const int j = tile_j[r];
+      const bool ok = j < N;
+      cp_async_16(kb + swz(r, c, S::kRowChunks), Kg + (size_t)(ok ? j : 0) * D + c * 8, ok ? 16 : 0);
+      cp_async_16(vb + swz(r, c, S::kRowChunks), Vg + (size_t)(ok ? j : 0) * D + c * 8, ok ? 16 : 0);
     }
     cp_async_commit();
   }
@@ -304,7 +308,7 @@ bwd_dkv_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
     dv[i][0] = dv[i][1] = dv[i][2] = dv[i][3] = 0.f;
   }
   const int kr0 = warp * 16 + (lane >> 2);        // this thread's key rows kr0, kr0 + 8
-  const int j_a = j0 + kr0, j_b = j_a + 8;
+  const int j_a = tile_j[kr0], j_b = tile_j[kr0 + 8];
 
   for (int hh = 0; hh < G; ++hh) {
     const int h = g * G + hh;
@@ -313,17 +317,20 @@ bwd_dkv_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
     const int32_t* erow = evict + bh * N;
     const int e_a = j_a < N ? erow[j_a] : 0, e_b = j_b < N ? erow[j_b] : 0;
     const float dl_a = j_a < N ? drow[j_a] * kLog2e : 0.f, dl_b = j_b < N ? drow[j_b] * kLog2e : 0.f;
-    if (tid == 0) qmax_sh = 0;
+    if (tid == 0) { qmax_sh = 0; qmin_sh = N; }
     __syncthreads();
-    {
-      int mymax = 0;
-      if (e_a > j_a) mymax = max(mymax, e_a);
-      if (e_b > j_b) mymax = max(mymax, e_b);
-      for (int o = 16; o > 0; o >>= 1) mymax = max(mymax, __shfl_xor_sync(0xffffffffu, mymax, o));
-      if (lane == 0) atomicMax(&qmax_sh, mymax);
+    {   // the query rows [qmin, qmax) that select some key of the tile in this head
+      int mymax = 0, mymin = N;
+      if (e_a > j_a) { mymax = max(mymax, e_a); mymin = min(mymin, j_a); }
+      if (e_b > j_b) { mymax = max(mymax, e_b); mymin = min(mymin, j_b); }
+      for (int o = 16; o > 0; o >>= 1) {
+        mymax = max(mymax, __shfl_xor_sync(0xffffffffu, mymax, o));
+        mymin = min(mymin, __shfl_xor_sync(0xffffffffu, mymin, o));
+      }
+      if (lane == 0) { atomicMax(&qmax_sh, mymax); atomicMin(&qmin_sh, mymin); }
     }
     __syncthreads();
-    const int qmax = qmax_sh;
+    const int qmax = qmax_sh, j0 = qmin_sh;
     const uint16_t* Qh = Q + bh * N * D;
     const uint16_t* Gh = dO + bh * N * D;
     const float* lse = LSE + bh * N;
@@ -450,6 +457,39 @@ bwd_dkv_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
   }
 }
 
+// Key order of the dK/dV pass.  A tile of 64 keys walks every query row that selects one of its keys
+// in some head of the group, so tiles that mix long- and short-lived keys spend MMAs on masked pairs.
+// Within each window of 256 positions the keys are therefore ordered by their group lifetime
+// max_h e_j (longest first, then position); consecutive 64-entry runs of this order form the tiles.
+constexpr int kOrderWin = 256;
+
+__global__ void __launch_bounds__(kOrderWin)
+bwd_key_order_kernel(const int32_t* __restrict__ evict, int32_t* __restrict__ perm, int H, int G, int N) {
+  __shared__ uint32_t key[kOrderWin];
+  const int w0 = blockIdx.x * kOrderWin, bg = blockIdx.y, tid = threadIdx.x;
+  const int Hkv = H / G, b = bg / Hkv, g = bg % Hkv;
+  const int j = w0 + tid;
+  uint32_t k = 0xffffffffu;   // past N: last
+  if (j < N) {
+    int me = j;
+    for (int hh = 0; hh < G; ++hh) me = max(me, evict[((size_t)b * H + g * G + hh) * N + j]);
+    k = ((uint32_t)(N - me) << 16) | (uint32_t)j;   // ascending = lifetime end descending, then j
+  }
+  key[tid] = k;
+  __syncthreads();
+  for (int size = 2; size <= kOrderWin; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int partner = tid ^ stride;
+      if (partner > tid) {
+        const uint32_t a = key[tid], c = key[partner];
+        const bool up = (tid & size) == 0;
+        if ((a > c) == up) { key[tid] = c; key[partner] = a; }
+      }
+      __syncthreads();
+    }
+  if (j < N) perm[(size_t)bg * N + j] = (int32_t)(key[tid] & 0xffffu);
+}
+
 template <int D, typename OutT>
 cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                          const float* delta, const int32_t* evict, void* ws, const void* O,
@@ -467,11 +507,14 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
         Drow, (OutT*)dQ, P.H, P.G, P.N, P.n_blocks, P.list_cap, P.scale * kLog2e, P.scale);
   }
   {
+    int32_t* perm = ws_ptr<int32_t>(ws, P.off_bwd_perm);
+    bwd_key_order_kernel<<<dim3((P.N + kOrderWin - 1) / kOrderWin, P.B * P.Hkv), kOrderWin, 0, s>>>(
+        evict, perm, P.H, P.G, P.N);
     auto k = bwd_dkv_kernel<D, OutT>;
     const int smem = DkvSmem<D>::kBytes;
     { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
     k<<<dim3((P.N + 63) / 64, P.B * P.Hkv), kDkvThreads, smem, s>>>(
-        Q, K, V, dO, delta, evict, LSE, Drow, (OutT*)dK, (OutT*)dV, d_delta, P.H, P.G, P.N,
+        Q, K, V, dO, delta, evict, perm, LSE, Drow, (OutT*)dK, (OutT*)dV, d_delta, P.H, P.G, P.N,
         P.scale * kLog2e, P.scale);
   }
   return cudaGetLastError();

@@ -53,6 +53,7 @@ struct Plan {
   size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
   size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
+  size_t off_bwd_perm;                 // backward: key order of the dK/dV tiles [B, Hkv, N] i32
   size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
   size_t off_tw_keys;                  // top-w: sorted segments of composite keys [B, H, npad] u64
