@@ -294,7 +294,7 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
   // so that each lane keeps 4 KB of row loads of its warp in flight.
   constexpr int kStride = kDecThreads / 8;
   constexpr int kMaxIt = (kDecodeSplit + kStride - 1) / kStride;
-  constexpr int kChunk = 4;
+  constexpr int kChunk = 2;
   static_assert(kMaxIt % kChunk == 0, "chunks of keys per lane group");
   const int kfirst = k0 + warp * 4 + grp;
   int jl[kMaxIt];
