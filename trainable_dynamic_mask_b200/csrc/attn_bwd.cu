@@ -8,19 +8,17 @@
 // dQ = scale dS K, dK_g = scale sum_{h in g} dS_h^T Q_h, dV_g = sum_{h in g} P_h^T dO_h,
 // d delta_{h,j} = sum_t dS_tj (delta enters the scores additively, unscaled).
 //
-// Three kernels: rowdot (D), dq (query-major over each block's live-key list, like the forward,
-// so dQ needs no atomics) and dkv (key-major over 64-key position tiles: key j only receives
-// gradient from the queries t in [j, e_j), so each tile walks the query range
-// [tile start, max e_j) and masks per pair; the query heads of one KV group are summed in
-// registers, so dK and dV need no atomics either).  Tensor cores via mma.sync m16n8k16 bf16.
+// Kernels here: rowdot (D), the key order, and dkv (key-major over 64-key tiles: key j only receives
+// gradient from the queries t in [j, e_j), so each tile walks the query range [min j, max e_j) and
+// masks per pair; the query heads of one KV group are summed in registers, so dK and dV need no
+// atomics; mma.sync m16n8k16 bf16).  dQ is query-major over each block's live-key list, like the
+// forward, so it needs no atomics either: the tcgen05 kernel of attn_bwd_tc.cu.
 #include <limits.h>
 
 #include "common.cuh"
 
 namespace dma {
 namespace {
-
-constexpr int kBK = 64;
 
 // ---------------------------------------------------------------- D = rowsum(dO * O)
 template <typename OT>
@@ -35,200 +33,6 @@ __global__ void bwd_rowdot_kernel(const OT* __restrict__ O, const uint16_t* __re
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (lane == 0) Drow[r] = acc;
-}
-
-// ---------------------------------------------------------------- dQ
-constexpr int kDqThreads = 256;
-
-template <int D>
-struct DqSmem {
-  static constexpr int kRowChunks = D / 8;
-  static constexpr int kQBytes = kBlockQ * D * 2;
-  static constexpr int kKVBytes = kBK * D * 2;
-  static constexpr int kOffDO = kQBytes;
-  static constexpr int kOffK = kOffDO + kQBytes;
-  static constexpr int kOffV = kOffK + 2 * kKVBytes;
-  static constexpr int kOffMeta = kOffV + 2 * kKVBytes;
-  static constexpr int kBytes = kOffMeta + 2 * 3 * kBK * 4;
-};
-
-template <int D, int OffK, int OffV, int OffMeta, int NThreads>
-DMA_DEVINL void bwd_load_tile(unsigned char* sm, int stage, int tile, const int32_t* list, int n_live,
-                              const uint16_t* Kg, const uint16_t* Vg, const float* drow,
-                              const int32_t* erow) {
-  constexpr int kRowChunks = D / 8;
-  constexpr int kKVBytes = kBK * D * 2;
-  constexpr int kTPR = NThreads / kBK;                       // threads per key row
-  constexpr int kChunksPerThread = kRowChunks / kTPR;
-  const int tid = threadIdx.x;
-  const int r = tid / kTPR;
-  const int c0 = (tid % kTPR) * kChunksPerThread;
-  const int li = tile * kBK + r;
-  const int j = li < n_live ? list[li] : -1;
-  const uint32_t kbase = smem_u32(sm + OffK + stage * kKVBytes);
-  const uint32_t vbase = smem_u32(sm + OffV + stage * kKVBytes);
-  const uint16_t* ksrc = Kg + (size_t)(j < 0 ? 0 : j) * D;
-  const uint16_t* vsrc = Vg + (size_t)(j < 0 ? 0 : j) * D;
-  const int nbytes = j < 0 ? 0 : 16;
-#pragma unroll
-  for (int u = 0; u < kChunksPerThread; ++u) {
-    const int c = c0 + u;
-    cp_async_16(kbase + swz(r, c, kRowChunks), ksrc + c * 8, nbytes);
-    cp_async_16(vbase + swz(r, c, kRowChunks), vsrc + c * 8, nbytes);
-  }
-  if (c0 == 0) {
-    int32_t* mj = reinterpret_cast<int32_t*>(sm + OffMeta) + stage * 3 * kBK;
-    float* md = reinterpret_cast<float*>(mj + kBK);
-    int32_t* me = mj + 2 * kBK;
-    mj[r] = j < 0 ? INT_MAX : j;
-    md[r] = j < 0 ? 0.f : drow[j] * kLog2e;
-    me[r] = j < 0 ? 0 : erow[j];
-  }
-}
-
-template <int D, typename OutT>
-__global__ void __launch_bounds__(kDqThreads, 1)
-bwd_dq_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
-              const uint16_t* __restrict__ V, const uint16_t* __restrict__ dO,
-              const float* __restrict__ delta, const int32_t* __restrict__ evict,
-              const int32_t* __restrict__ counts, const int32_t* __restrict__ lists,
-              const float* __restrict__ LSE, const float* __restrict__ Drow, OutT* __restrict__ dQ,
-              int H, int G, int N, int n_blocks, int list_cap, float scale_log2, float scale) {
-  using S = DqSmem<D>;
-  extern __shared__ __align__(128) unsigned char sm[];
-  const int kb = n_blocks - 1 - (int)blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh % H, g = h / G, Hkv = H / G;
-  const int t0 = kb * kBlockQ;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int32_t* cnt = counts + ((size_t)bh * n_blocks + kb) * 2;
-  const int n_full = cnt[0], n_live = cnt[1];
-  const int32_t* list = lists + ((size_t)bh * n_blocks + kb) * list_cap;
-  const uint16_t* Kg = K + (size_t)(b * Hkv + g) * N * D;
-  const uint16_t* Vg = V + (size_t)(b * Hkv + g) * N * D;
-  const float* drow = delta + (size_t)bh * N;
-  const int32_t* erow = evict + (size_t)bh * N;
-  {
-    const uint16_t* Qb = Q + ((size_t)bh * N + t0) * D;
-    const uint16_t* Gb = dO + ((size_t)bh * N + t0) * D;
-    const uint32_t qbase = smem_u32(sm), gbase = smem_u32(sm + S::kOffDO);
-    for (int i = tid; i < kBlockQ * S::kRowChunks; i += kDqThreads) {
-      const int r = i / S::kRowChunks, c = i % S::kRowChunks;
-      const bool ok = t0 + r < N;
-      cp_async_16(qbase + swz(r, c, S::kRowChunks), Qb + (size_t)(ok ? r : 0) * D + c * 8, ok ? 16 : 0);
-      cp_async_16(gbase + swz(r, c, S::kRowChunks), Gb + (size_t)(ok ? r : 0) * D + c * 8, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  }
-  const int n_tiles = (n_live + kBK - 1) / kBK;
-  if (n_tiles > 0)
-    bwd_load_tile<D, S::kOffK, S::kOffV, S::kOffMeta, kDqThreads>(sm, 0, 0, list, n_live, Kg, Vg, drow, erow);
-  cp_async_commit();
-
-  const int qr0 = warp * 16 + (lane >> 2);
-  const int tq0 = t0 + qr0, tq1 = tq0 + 8;
-  const float lse0 = tq0 < N ? LSE[(size_t)bh * N + tq0] * kLog2e : 0.f;
-  const float lse1 = tq1 < N ? LSE[(size_t)bh * N + tq1] * kLog2e : 0.f;
-  const float D0 = tq0 < N ? Drow[(size_t)bh * N + tq0] : 0.f;
-  const float D1 = tq1 < N ? Drow[(size_t)bh * N + tq1] : 0.f;
-  float dq[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) dq[i][0] = dq[i][1] = dq[i][2] = dq[i][3] = 0.f;
-
-  for (int it = 0; it < n_tiles; ++it) {
-    const int stage = it & 1;
-    if (it + 1 < n_tiles) {
-      bwd_load_tile<D, S::kOffK, S::kOffV, S::kOffMeta, kDqThreads>(sm, stage ^ 1, it + 1, list, n_live, Kg,
-                                                                   Vg, drow, erow);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t qbase = smem_u32(sm), gbase = smem_u32(sm + S::kOffDO);
-    const uint32_t kbase = smem_u32(sm + S::kOffK + stage * S::kKVBytes);
-    const uint32_t vbase = smem_u32(sm + S::kOffV + stage * S::kKVBytes);
-    const int32_t* mj = reinterpret_cast<const int32_t*>(sm + S::kOffMeta) + stage * 3 * kBK;
-    const float* md = reinterpret_cast<const float*>(mj + kBK);
-    const int32_t* me = mj + 2 * kBK;
-
-    float s[kBK / 8][4], dp[kBK / 8][4];
-#pragma unroll
-    for (int i = 0; i < kBK / 8; ++i) {
-      s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-      dp[i][0] = dp[i][1] = dp[i][2] = dp[i][3] = 0.f;
-    }
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t qa[4], ga[4];
-      ldmatrix_x4(qbase + swz(warp * 16 + (lane & 15), 2 * kk + (lane >> 4), S::kRowChunks), qa[0], qa[1],
-                  qa[2], qa[3]);
-      ldmatrix_x4(gbase + swz(warp * 16 + (lane & 15), 2 * kk + (lane >> 4), S::kRowChunks), ga[0], ga[1],
-                  ga[2], ga[3]);
-#pragma unroll
-      for (int np = 0; np < kBK / 16; ++np) {
-        const int rr = np * 16 + ((lane >> 4) << 3) + (lane & 7), cc = 2 * kk + ((lane >> 3) & 1);
-        uint32_t r0, r1, r2, r3;
-        ldmatrix_x4(kbase + swz(rr, cc, S::kRowChunks), r0, r1, r2, r3);
-        mma_bf16_16816(s[2 * np], qa, r0, r1);
-        mma_bf16_16816(s[2 * np + 1], qa, r2, r3);
-        ldmatrix_x4(vbase + swz(rr, cc, S::kRowChunks), r0, r1, r2, r3);
-        mma_bf16_16816(dp[2 * np], ga, r0, r1);
-        mma_bf16_16816(dp[2 * np + 1], ga, r2, r3);
-      }
-    }
-    const bool full_tile = (it + 1) * kBK <= n_full;
-#pragma unroll
-    for (int nt = 0; nt < kBK / 8; ++nt) {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int col = nt * 8 + (lane & 3) * 2 + u;
-        const float dl = md[col];
-        float p0 = fast_exp2(fmaf(s[nt][u], scale_log2, dl) - lse0);
-        float p1 = fast_exp2(fmaf(s[nt][2 + u], scale_log2, dl) - lse1);
-        if (!full_tile) {
-          const int jj = mj[col], ee = me[col];
-          if (!(jj <= tq0 && tq0 < ee)) p0 = 0.f;
-          if (!(jj <= tq1 && tq1 < ee)) p1 = 0.f;
-        }
-        s[nt][u] = p0 * (dp[nt][u] - D0);          // dS
-        s[nt][2 + u] = p1 * (dp[nt][2 + u] - D1);
-      }
-    }
-#pragma unroll
-    for (int kk = 0; kk < kBK / 16; ++kk) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-      for (int dn = 0; dn < D / 16; ++dn) {
-        uint32_t r0, r1, r2, r3;
-        ldmatrix_x4_trans(kbase + swz(kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3), 2 * dn + (lane >> 4),
-                                      S::kRowChunks),
-                          r0, r1, r2, r3);
-        mma_bf16_16816(dq[2 * dn], pa, r0, r1);
-        mma_bf16_16816(dq[2 * dn + 1], pa, r2, r3);
-      }
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
-  OutT* out = dQ + ((size_t)bh * N) * D;
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) {
-    const int col = i * 8 + (lane & 3) * 2;
-    if (tq0 < N) {
-      store_from_f32(out + (size_t)tq0 * D + col, dq[i][0] * scale);
-      store_from_f32(out + (size_t)tq0 * D + col + 1, dq[i][1] * scale);
-    }
-    if (tq1 < N) {
-      store_from_f32(out + (size_t)tq1 * D + col, dq[i][2] * scale);
-      store_from_f32(out + (size_t)tq1 * D + col + 1, dq[i][3] * scale);
-    }
-  }
 }
 
 // ---------------------------------------------------------------- dK, dV, d delta
@@ -499,12 +303,8 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
   const size_t rows = (size_t)P.B * P.H * P.N;
   bwd_rowdot_kernel<OutT><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const OutT*)O, dO, Drow, rows, D);
   {
-    auto k = bwd_dq_kernel<D, OutT>;
-    const int smem = DqSmem<D>::kBytes;
-    { cudaError_t ea = ensure_smem_limit(k, smem); if (ea != cudaSuccess) return ea; }
-    k<<<dim3(P.n_blocks, P.B * P.H), kDqThreads, smem, s>>>(
-        Q, K, V, dO, delta, evict, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists), LSE,
-        Drow, (OutT*)dQ, P.H, P.G, P.N, P.n_blocks, P.list_cap, P.scale * kLog2e, P.scale);
+    cudaError_t e = launch_bwd_dq_tc(P, Q, K, V, dO, delta, evict, ws, LSE, Drow, dQ, s);
+    if (e != cudaSuccess) return e;
   }
   {
     int32_t* perm = ws_ptr<int32_t>(ws, P.off_bwd_perm);

@@ -36,7 +36,7 @@
 
 #include <mutex>
 
-#include "tc.cuh"
+#include "tc_ops.cuh"
 
 namespace dma {
 namespace {
@@ -80,120 +80,10 @@ struct TcBars {
   int merge_old[2];   // per softmax warpgroup: arrivals seen by its unit's merge counter
 };
 
-DMA_DEVINL void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n" ::"r"(
-                   smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-// Four rows (r0..r3) x 64 columns starting at column `col` of a 2-D tensor map, written as four
-// consecutive 128-byte rows at `dst` (the map's 128-byte swizzle applies); completion is counted
-// in bytes on `bar`.
-DMA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r0, int r1, int r2, int r3,
-                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Warp-uniform bounded wait (every lane of the warp calls it).
-DMA_DEVINL bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status, int code) {
-  return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag, status, code));
-}
-
-// Wait that ignores the abort flag, for draining copies in flight after an abort (bounded).
-DMA_DEVINL void drain_wait(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!tc::mbar_try_wait(bar, parity) && clock64() - t0 < 200000000LL) {
-  }
-}
-
 // Named barrier of one softmax warpgroup (ids 1 and 2; 0 is __syncthreads).
 DMA_DEVINL void group_sync(int h) {
   if (h == 0) asm volatile("bar.sync 1, 128;\n" ::: "memory");
   else asm volatile("bar.sync 2, 128;\n" ::: "memory");
-}
-
-template <int R> DMA_DEVINL void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R)); }
-template <int R> DMA_DEVINL void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R)); }
-
-// ---- packed f32x2 arithmetic (two lanes of FP32 work per instruction on sm_100)
-DMA_DEVINL uint64_t f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-DMA_DEVINL void f2_split(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
-DMA_DEVINL uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-DMA_DEVINL uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-DMA_DEVINL uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-DMA_DEVINL float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// 2^x for a pair of x <= ~8 on the FMA pipe: x = i + f with i = round(x), f in [-1/2, 1/2];
-// 2^f ~ 1 + f (c1 + f (c2 + f c3)), a cubic fitted here for minimum relative error on [-1/2, 1/2]
-// (max 1.02e-4, far below bf16's half ulp 2^-9, the precision P is stored in); i is added to the
-// exponent field.  x is clamped at -127, where f = 0, p = 1 exactly and the exponent sum wraps to
-// +0: masked entries (x = -inf) give exactly 0, as the MUFU path does.  Round-to-nearest uses the
-// 1.5 * 2^23 shift: the integer lands in the low mantissa bits of x + 1.5 * 2^23.
-DMA_DEVINL void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
-  constexpr float c1 = 0.6932829022407532f, c2 = 0.24221068620681763f, c3 = 0.05500871315598488f;
-  x0 = fmaxf(x0, -127.f);
-  x1 = fmaxf(x1, -127.f);
-  const uint64_t x = f2(x0, x1);
-  const uint64_t r = f2_add(x, f2(kShift, kShift));
-  const uint64_t f = f2_sub(x, f2_sub(r, f2(kShift, kShift)));
-  uint64_t p = f2_fma(f, f2(c3, c3), f2(c2, c2));
-  p = f2_fma(f, p, f2(c1, c1));
-  p = f2_fma(f, p, f2(1.f, 1.f));
-  float r0, r1, q0, q1;
-  f2_split(r, r0, r1);
-  f2_split(p, q0, q1);
-  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(r0) << 23));
-  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(r1) << 23));
-}
-
-// tcgen05.mma (kind::f16, A and B from shared memory) with both descriptors advanced by OFF / 16
-// inside the asm block: the 8 K steps then need no live descriptor registers each.
-template <uint32_t OFF>
-DMA_DEVINL void mma_ss_at(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
-      "add.s64 a, %1, %5;\n\t"
-      "add.s64 b, %2, %5;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(OFF >> 4));
-}
-// tcgen05.mma with A = P from TMEM column a_tmem + 8 KK and B = V at descriptor + KK * 2048 / 16.
-template <int KK>
-DMA_DEVINL void mma_ts_at(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "add.s64 b, %2, %5;\n\t"
-      "add.u32 a, %1, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(KK * 2048 / 16), "n"(KK * 8));
 }
 
 template <int KK, int NK>
@@ -236,22 +126,6 @@ DMA_DEVINL void issue_pv(uint32_t tmem, int half, uint64_t dv, bool first, uint6
   tc::commit(done);
 }
 
-// 32 consecutive outputs of a row (16-byte stores).
-DMA_DEVINL void store_row32(uint16_t* dst, const float (&v)[32]) {
-#pragma unroll
-  for (int u = 0; u < 32; u += 8) {
-    uint4 w;
-    w.x = pack_bf16x2(v[u], v[u + 1]);
-    w.y = pack_bf16x2(v[u + 2], v[u + 3]);
-    w.z = pack_bf16x2(v[u + 4], v[u + 5]);
-    w.w = pack_bf16x2(v[u + 6], v[u + 7]);
-    *reinterpret_cast<uint4*>(dst + u) = w;
-  }
-}
-DMA_DEVINL void store_row32(float* dst, const float (&v)[32]) {
-#pragma unroll
-  for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
-}
 DMA_DEVINL int ld_acquire(const int32_t* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -514,7 +388,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 #pragma unroll
         for (int c = 0; c < kTcBK / 32; ++c) tc::tmem_ld32(tS + c * 32, sr[c]);
         // this tile's metadata: entry r from this thread, the others through the shared buffer
-        float* buf = meta + (i & 1) * 3 * kTcBK;
+        float* buf = meta + (tt & 1) * 3 * kTcBK;   // by the CTA's tile count: alternates across items too
         buf[r] = dl_n;
         reinterpret_cast<int32_t*>(buf)[kTcBK + r] = jj_n;
         reinterpret_cast<int32_t*>(buf)[2 * kTcBK + r] = ln_n;
@@ -741,50 +615,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   __syncthreads();
   tc::fence_after();
   if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
-}
-
-// ---------------------------------------------------------------- host side: tensor maps
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// SMs of the current device (cached per device).
-int sm_count() {
-  static std::mutex mu;
-  static int count[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  std::lock_guard<std::mutex> lock(mu);
-  if (count[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    count[dev] = n;
-  }
-  return count[dev];
-}
-
-// 2-D view [rows, d] of a row-major bf16 tensor; boxes of 64 columns x 1 row (the gather4 form),
-// 128-byte swizzle.
-bool make_row_map(CUtensorMap* map, const void* base, uint64_t rows, int d) {
-  auto enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D, typename OutT>

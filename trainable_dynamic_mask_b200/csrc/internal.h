@@ -77,6 +77,12 @@ template <typename T> inline T* ws_ptr(void* ws, size_t off) {
   return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
 }
 
+// ---------------------------------------------------------------- host helpers (tmap.cu)
+// 2-D view [rows, d] of a row-major bf16 tensor for TMA gather4: boxes of 64 columns x 1 row,
+// 128-byte swizzle.  `map` must point to a CUtensorMap (128 bytes, 64-byte aligned).
+bool make_row_map(void* map, const void* base, uint64_t rows, int d);
+int sm_count();   // SMs of the current device
+
 // ---------------------------------------------------------------- launchers (cudaError_t)
 cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             float* delta, float* x_save, cudaStream_t s);
@@ -97,6 +103,9 @@ cudaError_t launch_attn_bwd(const Plan& P, const uint16_t* Q, const uint16_t* K,
                             const uint16_t* V, const float* delta, const int32_t* evict,
                             void* ws, const void* O, const float* LSE, const uint16_t* dO16,
                             void* dQ, void* dK, void* dV, float* d_delta, cudaStream_t s);
+cudaError_t launch_bwd_dq_tc(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const uint16_t* dO, const float* delta, const int32_t* evict, void* ws,
+                             const float* LSE, const float* Drow, void* dQ, cudaStream_t s);
 cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             const float* x_save, const float* delta, const float* d_delta,
                             float* dDelta, float* dA, float* dV_gate, void* ws, cudaStream_t s);
