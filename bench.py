@@ -414,7 +414,7 @@ def leg_train(args, world, torch, dma, peaks):
             "fwd_ms": round(t_f, 4), "bwd_ms": round(t_b, 4),
             "fwd_tflops": round(ff / (t_f * 1e-3) / 1e12, 2), "bwd_tflops": round(fb / (t_b * 1e-3) / 1e12, 2),
             "bwd_frac_of_peak": round(fb / (t_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
-            "gpu_launches": 14 * n}   # forward 7, attention backward 3, gate backward 4
+            "gpu_launches": 17 * n}   # forward 7, attention backward 6, gate backward 4
 
 
 # ---------------------------------------------------------------- the CPU oracle

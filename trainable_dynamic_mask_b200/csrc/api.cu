@@ -155,7 +155,13 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_fml = take((size_t)R.sched.n_slots * 2 * 2 * kBlockQ * sizeof(float));
     R.off_fcnt = take(BH * R.n_pairs * 4 * sizeof(int32_t));
     R.off_rowD = take(BH * R.Nq * sizeof(float));
-    R.off_bwd_perm = take((size_t)R.B * R.Hkv * R.N * sizeof(int32_t));
+    {
+      const size_t n_slots = BH * ((R.N + 1023) / 1024) * 8;   // windows of 1024 keys, tiles of 128
+      R.off_dkv_perm = take(BH * R.N * sizeof(int32_t));
+      R.off_dkv_slots = take(n_slots * 4 * sizeof(int32_t));
+      R.off_dkv_items = take((n_slots + 1) * sizeof(int32_t));
+      R.off_dkv_part = take(2 * BH * R.N * (size_t)R.d * sizeof(float));
+    }
     R.off_tw_p = take(BH * R.N * sizeof(int32_t));
     R.off_tw_rank = take(BH * R.N * sizeof(int32_t));
     R.off_tw_T = take(BH * (R.n_blocks + 1) * sizeof(int32_t));

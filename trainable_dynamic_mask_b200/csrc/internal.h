@@ -53,7 +53,9 @@ struct Plan {
   size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
   size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
-  size_t off_bwd_perm;                 // backward: key order of the dK/dV tiles [B, Hkv, N] i32
+  // backward dK/dV: per-head key order [B, H, N] i32, item records [n_slots] int4 {qlo, steps, keys,
+  // perm offset}, items by length [n_slots] + count i32, f32 partial dK_h, dV_h [2][B, H, N, d]
+  size_t off_dkv_perm, off_dkv_slots, off_dkv_items, off_dkv_part;
   size_t off_tw_p, off_tw_rank;        // top-w: rank -> position, position -> rank [B, H, N] i32
   size_t off_tw_T;                     // top-w: threshold ranks [B, H, n_blocks + 1] i32
   size_t off_tw_keys;                  // top-w: sorted segments of composite keys [B, H, npad] u64
@@ -81,6 +83,8 @@ template <typename T> inline T* ws_ptr(void* ws, size_t off) {
 // 2-D view [rows, d] of a row-major bf16 tensor for TMA gather4: boxes of 64 columns x 1 row,
 // 128-byte swizzle.  `map` must point to a CUtensorMap (128 bytes, 64-byte aligned).
 bool make_row_map(void* map, const void* base, uint64_t rows, int d);
+// 2-D view [rows, d] for TMA box loads: boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tile_map(void* map, const void* base, uint64_t rows, int d, int box_rows);
 int sm_count();   // SMs of the current device
 
 // ---------------------------------------------------------------- launchers (cudaError_t)
@@ -106,6 +110,10 @@ cudaError_t launch_attn_bwd(const Plan& P, const uint16_t* Q, const uint16_t* K,
 cudaError_t launch_bwd_dq_tc(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                              const uint16_t* dO, const float* delta, const int32_t* evict, void* ws,
                              const float* LSE, const float* Drow, void* dQ, cudaStream_t s);
+cudaError_t launch_bwd_dkv_tc(const Plan& P, const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                              const uint16_t* dO, const float* delta, const int32_t* evict, void* ws,
+                              const float* LSE, const float* Drow, void* dK, void* dV, float* d_delta,
+                              cudaStream_t s);
 cudaError_t launch_gate_bwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             const float* x_save, const float* delta, const float* d_delta,
                             float* dDelta, float* dA, float* dV_gate, void* ws, cudaStream_t s);

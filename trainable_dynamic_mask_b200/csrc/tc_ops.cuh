@@ -28,6 +28,16 @@ DMA_DEVINL void tma_gather4(uint32_t dst, const CUtensorMap* map, int col, int r
       : "memory");
 }
 
+// The box of a 2-D tensor map whose first element is (x = column, y = row), written to `dst` (the
+// map's swizzle applies); completion is counted in bytes on `bar`.  Rows past the tensor read 0.
+DMA_DEVINL void tma_tile_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Warp-uniform bounded wait (every lane of the warp calls it).
 DMA_DEVINL bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status, int code) {
   return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, abort_flag, status, code));

@@ -1,5 +1,5 @@
 // Host helpers of the tcgen05 kernels: the driver's tensor-map encoder (looked up once through the
-// runtime), 2-D bf16 row maps for TMA gathers, and the SM count of the current device.
+// runtime), 2-D bf16 row maps for TMA gathers and tile maps for TMA box loads, and the SM count of the current device.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,6 +46,20 @@ bool make_row_map(void* map_out, const void* base, uint64_t rows, int d) {
   cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)rows};
   cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
   cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D view [rows, d] of a row-major bf16 tensor; boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_tile_map(void* map_out, const void* base, uint64_t rows, int d, int box_rows) {
+  CUtensorMap* map = static_cast<CUtensorMap*>(map_out);
+  auto enc = encode_fn();
+  if (enc == nullptr || box_rows < 1 || box_rows > 256) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
