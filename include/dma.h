@@ -86,7 +86,7 @@ typedef enum {
  *   dtype  a dma_dtype_t
  *
  * Limits of this implementation (DMA_ERR_UNSUPPORTED beyond them): prefill/training
- * N <= 16384; decode N <= 1<<24; B*H <= 65535; d in {64, 128}.
+ * N <= 16384; decode N <= 1<<24 and min(w, N) <= 4096 * d; B*H <= 65535; d in {64, 128}.
  */
 typedef struct {
   int32_t B, H, Hkv, N, Nq, d, w;

@@ -134,6 +134,8 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   R.n_pairs = (R.N + kPairQ - 1) / kPairQ;
   R.sel_len = minwn;
   R.n_split = (R.sel_len + kDecodeSplit - 1) / kDecodeSplit;
+  // decode combines its splits' (m, l) in shared memory, within kDecodeSplit * d * 2 bytes
+  if (R.decode && (size_t)R.n_split * 2 * sizeof(float) > (size_t)kDecodeSplit * R.d * 2) return DMA_ERR_UNSUPPORTED;
   R.n_slices = (R.N + kGateSlice - 1) / kGateSlice;
 
   size_t off = 0;

@@ -12,7 +12,7 @@ namespace dma {
 constexpr int kBlockQ = DMA_BLOCK_Q;   // query rows per block of the mask encoding
 constexpr int kPairQ = 2 * kBlockQ;    // query rows per attention-forward work item
 constexpr int kTopwMaxN = 16384;      // prefill/training selection keeps a whole row in SMEM
-constexpr int kDecodeSplit = 256;      // selected keys per decode split
+constexpr int kDecodeSplit = 256;      // selected keys per decode split (one per thread)
 constexpr int kGateSlice = 512;        // positions per partial sum of dDelta
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
