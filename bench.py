@@ -296,10 +296,11 @@ def run_ours(args, world, rank):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
     }
-    if not args.no_legs:
-        line["legs"] = {"decode": leg_decode(args, world, torch, dma, peaks),
-                        "train": leg_train(args, world, torch, dma, peaks)}
-        line["gpu_launches"] += line["legs"]["decode"]["gpu_launches"] + line["legs"]["train"]["gpu_launches"]
+    legs = [] if args.no_legs else [x for x in args.legs.split(",") if x]
+    if legs:
+        run = {"decode": leg_decode, "train": leg_train}
+        line["legs"] = {name: run[name](args, world, torch, dma, peaks) for name in legs}
+        line["gpu_launches"] += sum(leg["gpu_launches"] for leg in line["legs"].values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
     return line
@@ -520,6 +521,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-legs", action="store_true", help="skip the decode and training legs")
+    ap.add_argument("--legs", default="decode,train", help="comma-separated legs to run: decode, train")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)

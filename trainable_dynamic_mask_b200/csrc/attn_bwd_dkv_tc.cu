@@ -25,9 +25,13 @@
 //               dS^T (bf16) are written back over the columns of S^T and dP^T they were read from;
 //               at the end of an item, warps 0-3 write dK (x scale) and warps 4-7 dV, and each
 //               half adds its row sums of dS^T to d delta (two f32 adds onto 0: exact in any order);
-//   warp 8      TMEM allocation; one thread issues S^T = K Q^T and dP^T = V dO^T (operands
-//               in shared memory), then dV += P^T dO and dK += dS^T Q (A from TMEM, B read N-major);
-//   warps 9, 10 gather the item's K and V rows (TMA tile::gather4), double-buffered across items;
+//   warp 8      TMEM allocation; one thread issues S^T = K Q^T and dP^T = V dO^T (operands in
+//               shared memory);
+//   warp 10     one thread issues dV += P^T dO and dK += dS^T Q (A from TMEM, B read N-major).
+//               Two issuing threads on different SM sub-partitions: one thread's tcgen05.mma issue
+//               rate drops well below the tensor pipe's rate while the elementwise warps keep its
+//               sub-partition busy, and each thread's commits track only its own MMAs;
+//   warp 9      gathers the item's K and V rows (TMA tile::gather4), double-buffered across items;
 //   warp 11     loads the Q and dO tiles of each step (TMA tiles of 64 rows), three stages.
 // TMEM: S^T buffers at columns 0 and 128, dP^T at 64 and 192 (64 columns each; step T uses buffer
 // T % 2, so the S^T/dP^T products of step T + 1 run while step T is elementwise), dK [256, 256 + D),
@@ -42,7 +46,7 @@ namespace {
 
 constexpr int kDkThreads = 384;
 constexpr int kDkMmaWarp = 8;
-constexpr int kDkKWarp = 9, kDkVWarp = 10, kDkQWarp = 11;
+constexpr int kDkKVWarp = 9, kDkGradWarp = 10, kDkQWarp = 11;
 constexpr int kDkBK = 128;        // keys per item
 constexpr int kDkBQ = 64;         // queries per step
 constexpr int kDkQStages = 3;     // Q / dO stages
@@ -271,7 +275,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       bar.abort_flag = 1;
     }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bar.kv_full[i], 64);
+      tc::mbar_init(&bar.kv_full[i], 32);
       tc::mbar_init(&bar.kv_empty[i], 1);
       tc::mbar_init(&bar.s_full[i], 1);
       tc::mbar_init(&bar.ds_full[i], 256);
@@ -279,11 +283,11 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
     for (int i = 0; i < kDkQStages; ++i) {
       tc::mbar_init(&bar.qd_full[i], 1);
-      tc::mbar_init(&bar.qd_empty[i], 1);
+      tc::mbar_init(&bar.qd_empty[i], 2);   // both MMA issuers read the stage
     }
     tc::mbar_init(&bar.acc_full, 1);
     tc::mbar_init(&bar.acc_empty, 256);
-    tc::mbar_init(&bar.drain, 1);
+    tc::mbar_init(&bar.drain, 2);
     tc::fence_mbar_init();
   }
   if (warp == kDkMmaWarp) {
@@ -308,11 +312,8 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
   int4 rec;
   int bh;
 
-  if (warp == kDkKWarp || warp == kDkVWarp) {
-    // ------------------------------------------------------------ K or V rows of each item (gather4)
-    const bool kside = warp == kDkKWarp;
-    const CUtensorMap* map = kside ? &kmap : &vmap;
-    const int base = kside ? S::kK : S::kV;
+  if (warp == kDkKVWarp) {
+    // ------------------------------------------------------------ K and V rows of each item (gather4)
     int n = 0;
     bool ok = !*abort_flag;
     for (int r = 0; ok && item_at(r, rec, bh); ++r, ++n) {
@@ -329,11 +330,14 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const int li = 4 * lane + u;
         rr[u] = kvrow0 + (li < rec.z ? perm[rec.w + li] : 0);
       }
-      mbar_arrive_expect_tx(&bar.kv_full[buf], 4 * kRowBytes);
+      mbar_arrive_expect_tx(&bar.kv_full[buf], 8 * kRowBytes);
 #pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf)
-        tma_gather4(smem_u32(sm + base + buf * S::kKV) + hf * (kDkBK * 128) + lane * 512, map, hf * 64, rr[0], rr[1],
-                    rr[2], rr[3], &bar.kv_full[buf]);
+      for (int hf = 0; hf < D / 64; ++hf) {
+        tma_gather4(smem_u32(sm + S::kK + buf * S::kKV) + hf * (kDkBK * 128) + lane * 512, &kmap, hf * 64, rr[0],
+                    rr[1], rr[2], rr[3], &bar.kv_full[buf]);
+        tma_gather4(smem_u32(sm + S::kV + buf * S::kKV) + hf * (kDkBK * 128) + lane * 512, &vmap, hf * 64, rr[0],
+                    rr[1], rr[2], rr[3], &bar.kv_full[buf]);
+      }
     }
     if (!ok)
       for (int m = n >= 2 ? n - 2 : 0; m < n; ++m) drain_wait(&bar.kv_full[m & 1], (m >> 1) & 1);
@@ -367,28 +371,11 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           drain_wait(&bar.qd_full[m % kDkQStages], (m / kDkQStages) & 1);
     }
   } else if (warp == kDkMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer (one thread)
+    // ------------------------------------------------------------ S^T and dP^T issuer (one thread)
     if (lane == 0) {
       constexpr uint32_t id_sdp = tc::idesc_bf16(128, kDkBQ, false, false);
-      constexpr uint32_t id_grad = tc::idesc_bf16(128, D, false, true);
       int T = 0, n = 0;
       bool ok = !*abort_flag;
-      // dV += P^T(U) dO(U), dK += dS^T(U) Q(U); `first` starts the item's accumulators, which the
-      // previous item's epilogue must have read
-      auto issue_grad = [&](int U, bool first) -> bool {
-        const int b = U & 1, st = U % kDkQStages;
-        if (!tc::mbar_wait(&bar.ds_full[b], (U >> 1) & 1, abort_flag, status, kErrDkDS)) return false;
-        if (first && n >= 1 && !tc::mbar_wait(&bar.acc_empty, (n - 1) & 1, abort_flag, status, kErrDkAcc))
-          return false;
-        tc::fence_after();
-        const uint64_t bdo = tc::sdesc(smem_u32(sm + S::kdO + st * S::kQT), kDkBQ * 128, 1024);
-        const uint64_t bq = tc::sdesc(smem_u32(sm + S::kQ + st * S::kQT), kDkBQ * 128, 1024);
-        DkGradSteps<0>::run(tmem + kDkDV, tmem + b * kDkBuf + kDkS, bdo, id_grad, first ? 0u : 1u);
-        DkGradSteps<0>::run(tmem + kDkDK, tmem + b * kDkBuf + kDkDP, bq, id_grad, first ? 0u : 1u);
-        tc::commit(&bar.mma_done[b]);
-        tc::commit(&bar.qd_empty[st]);
-        return true;
-      };
       for (int r = 0; ok && item_at(r, rec, bh); ++r, ++n) {
         const int kvb = n & 1;
         if (!(ok = tc::mbar_wait(&bar.kv_full[kvb], (n >> 1) & 1, abort_flag, status, kErrDkKV))) break;
@@ -398,7 +385,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         for (int i = 0; i < steps; ++i) {
           const int U = T + i, b = U & 1, st = U % kDkQStages;
           if (!(ok = tc::mbar_wait(&bar.qd_full[st], (U / kDkQStages) & 1, abort_flag, status, kErrDkQ))) break;
-          // buffer b last held step U - 2, whose gradient products were issued before this point
+          // buffer b last held step U - 2: its gradient products (the other issuer) must be done
           if (U >= 2 && !(ok = tc::mbar_wait(&bar.mma_done[b], ((U >> 1) - 1) & 1, abort_flag, status, kErrDkDone)))
             break;
           tc::fence_after();
@@ -407,11 +394,40 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           DkSdpSteps<0, D / 16>::run(tmem + b * kDkBuf + kDkS, ak, bq, id_sdp);
           DkSdpSteps<0, D / 16>::run(tmem + b * kDkBuf + kDkDP, av, bdo, id_sdp);
           tc::commit(&bar.s_full[b]);
+          tc::commit(&bar.qd_empty[st]);
           if (i + 1 == steps) tc::commit(&bar.kv_empty[kvb]);   // K and V of the item read for the last time
-          if (i >= 1 && !(ok = issue_grad(U - 1, i == 1))) break;
         }
         if (!ok) break;
-        if (!(ok = issue_grad(T + steps - 1, steps == 1))) break;
+        T += steps;
+      }
+      tc::commit(&bar.drain);
+      drain_wait(&bar.drain, 0);
+    }
+    __syncwarp();
+  } else if (warp == kDkGradWarp) {
+    // ------------------------------------------------------------ dV and dK issuer (one thread)
+    if (lane == 0) {
+      constexpr uint32_t id_grad = tc::idesc_bf16(128, D, false, true);
+      int T = 0, n = 0;
+      bool ok = !*abort_flag;
+      for (int r = 0; ok && item_at(r, rec, bh); ++r, ++n) {
+        const int steps = rec.y;
+        for (int i = 0; i < steps; ++i) {
+          // dV += P^T(U) dO(U), dK += dS^T(U) Q(U); the first step of an item starts the accumulators,
+          // which the previous item's epilogue must have read
+          const int U = T + i, b = U & 1, st = U % kDkQStages;
+          if (!(ok = tc::mbar_wait(&bar.ds_full[b], (U >> 1) & 1, abort_flag, status, kErrDkDS))) break;
+          if (i == 0 && n >= 1 && !(ok = tc::mbar_wait(&bar.acc_empty, (n - 1) & 1, abort_flag, status, kErrDkAcc)))
+            break;
+          tc::fence_after();
+          const uint64_t bdo = tc::sdesc(smem_u32(sm + S::kdO + st * S::kQT), kDkBQ * 128, 1024);
+          const uint64_t bq = tc::sdesc(smem_u32(sm + S::kQ + st * S::kQT), kDkBQ * 128, 1024);
+          DkGradSteps<0>::run(tmem + kDkDV, tmem + b * kDkBuf + kDkS, bdo, id_grad, i == 0 ? 0u : 1u);
+          DkGradSteps<0>::run(tmem + kDkDK, tmem + b * kDkBuf + kDkDP, bq, id_grad, i == 0 ? 0u : 1u);
+          tc::commit(&bar.mma_done[b]);
+          tc::commit(&bar.qd_empty[st]);
+        }
+        if (!ok) break;
         tc::commit(&bar.acc_full);
         T += steps;
       }
