@@ -40,6 +40,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "DMA fwd kept-pair TFLOP/s & % bf16 peak; decode selected-KV GB/s vs HBM"
+# The pages' own speed claim, quoted beside our figures (context, not a target): page 1 (HF blog
+# "dmattn"), section "Practical Speed Improvements"; the pages name no hardware.
+PAGES_CLAIM = {"claim": "training: up to 10x speedup over standard attention for longer sequences; "
+                        "inference: gains compounding as sequence length increases",
+               "source": "Trainable Dynamic Mask Sparse Attention (HF blog dmattn), Practical Speed Improvements",
+               "hardware": "not stated"}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -233,6 +239,37 @@ def run_ours(args, world, rank):
     achieved = flops / (attn_avg * 1e-3) / 1e12
     traffic = _traffic("attn_fwd_prefill", "attn_fwd_tc.cu")
 
+    # the same kernels with w = N (dense causal attention), timed the same way
+    wl_d = wl.with_(w=wl.N)
+    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, dtype="bf16")
+    ws_d = dma.alloc_workspace(p_d)
+    O_d, LSE_d = torch.empty_like(O), torch.empty_like(LSE)
+    with torch.cuda.stream(stream):
+        dma.gate(p_d, V, Dl, A, delta, None, ws_d, s_ptr)
+        dma.topk_mask(p_d, delta, evict, ws_d, s_ptr)
+        dma.attn_fwd(p_d, Q, K, V, delta, evict, ws_d, O_d, LSE_d, s_ptr)
+        stream.synchronize()
+        gda, gdb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gda, stream=stream):
+            dma.gate(p_d, V, Dl, A, delta, None, ws_d, s_ptr)
+            dma.topk_mask(p_d, delta, evict, ws_d, s_ptr)
+        with torch.cuda.graph(gdb, stream=stream):
+            dma.attn_fwd(p_d, Q, K, V, delta, evict, ws_d, O_d, LSE_d, s_ptr)
+    ga_s, gb_s = ga, gb
+    ga, gb = gda, gdb
+    timed(args.warmup)
+    n_d = max(5, min(args.steps, 100))
+    step_d, attn_d = timed(n_d)
+    ga, gb = ga_s, gb_s
+    step_d = _max_over_ranks(sum(step_d), world, torch) / n_d
+    attn_d = _max_over_ranks(sum(attn_d), world, torch) / n_d
+    flops_d = 4.0 * wl.d * wl_d.kept_pairs()
+    dense = {"w": wl.N, "kept_pairs": wl_d.kept_pairs(), "step_us": round(step_d * 1e3, 2),
+             "attn_us": round(attn_d * 1e3, 2), "attn_tflops": round(flops_d / (attn_d * 1e-3) / 1e12, 2),
+             "speedup_attn": round(attn_d / attn_avg, 3), "speedup_step": round(step_d / ms_per_step, 3),
+             "steps": n_d}
+    del ws_d, O_d, LSE_d
+
     # end to end through the public API: pinned host inputs in, O and LSE back to the host
     host = {n: torch.from_numpy(np.ascontiguousarray(I.bits[n]).view(np.int16)).view(torch.bfloat16).pin_memory()
             for n in ("Q", "K", "V", "Delta")}
@@ -295,6 +332,8 @@ def run_ours(args, world, rank):
                 "api": "trainable_dynamic_mask_b200.forward"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "dense_causal": dense,
+        "pages_claim": PAGES_CLAIM,
     }
     legs = [] if args.no_legs else [x for x in args.legs.split(",") if x]
     if legs:
@@ -354,6 +393,26 @@ def leg_decode(args, world, torch, dma, peaks):
     t_sel = _max_over_ranks(t_sel, world, torch) / n
     t_att = _max_over_ranks(t_att, world, torch) / n
     gbs = bytes_unique / (t_att * 1e-3) / 1e9
+    # the same kernels with w = L (every cached row attended), timed the same way
+    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, Nq=1, dtype="bf16")
+    ws_d = dma.alloc_workspace(p_d)
+    dma.topk_mask(p_d, delta, None, ws_d)
+    td = 0.0
+    n_d = 5
+    for i in range(2 + n_d):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dma.attn_fwd(p_d, Q, K, V, delta, None, ws_d, O, LSE)
+        b.record()
+        b.synchronize()
+        if i >= 2:
+            td += a.elapsed_time(b)
+    del ws_d
+    td = _max_over_ranks(td, world, torch) / n_d
+    bytes_d = wl.B * wl.Hkv * wl.N * 2 * wl.d * 2
+    dense = {"w": wl.N, "attn_us": round(td * 1e3, 2), "gbs": round(bytes_d / (td * 1e-3) / 1e9, 2),
+             "speedup_attn": round(td / t_att, 3), "steps": n_d}
     return {"metric": "decode selected-KV GB/s", "value": round(world * gbs, 2), "unit": "GB/s",
             "config": {"workload": "decode", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "L": wl.N, "d": wl.d, "w": wl.w},
             "attn_us": round(t_att * 1e3, 2), "select_us": round(t_sel * 1e3, 2),
@@ -361,6 +420,7 @@ def leg_decode(args, world, torch, dma, peaks):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "peak_kind": peaks["source"], "traffic": None,
                          "algorithmic_bytes": bytes_unique, "bytes_if_per_head": bytes_per_head},
+            "dense_causal": dense,
             "gpu_launches": 3 * n}
 
 
@@ -408,6 +468,33 @@ def leg_train(args, world, torch, dma, peaks):
     t_f = _max_over_ranks(t_f, world, torch) / n
     t_b = _max_over_ranks(t_b, world, torch) / n
     ff, fb = 4.0 * wl.d * pairs, 10.0 * wl.d * pairs
+    # the same kernels with w = N (dense causal), timed the same way
+    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, dtype="bf16")
+    ws_d = dma.alloc_workspace(p_d)
+    td_f = td_b = 0.0
+    n_d = 3
+    for i in range(2 + n_d):
+        flush.zero_()
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record()
+        dma.gate(p_d, V, Dl, A, delta, x, ws_d)
+        dma.topk_mask(p_d, delta, evict, ws_d)
+        dma.attn_fwd(p_d, Q, K, V, delta, evict, ws_d, O, LSE)
+        b.record()
+        dma.attn_bwd(p_d, Q, K, V, delta, evict, ws_d, O, LSE, dO, dQ, dK, dV, dd)
+        dma.gate_bwd(p_d, V, Dl, A, x, delta, dd, dDelta, dA, dVg, ws_d)
+        c.record()
+        c.synchronize()
+        if i >= 2:
+            td_f += a.elapsed_time(b)
+            td_b += b.elapsed_time(c)
+    del ws_d
+    td_f = _max_over_ranks(td_f, world, torch) / n_d
+    td_b = _max_over_ranks(td_b, world, torch) / n_d
+    pairs_d = wl.with_(w=wl.N).kept_pairs()
+    dense = {"w": wl.N, "kept_pairs": pairs_d, "fwd_ms": round(td_f, 4), "bwd_ms": round(td_b, 4),
+             "tflops": round(14.0 * wl.d * pairs_d / ((td_f + td_b) * 1e-3) / 1e12, 3),
+             "speedup_fwd_bwd": round((td_f + td_b) / (t_f + t_b), 3), "steps": n_d}
     return {"metric": "train fwd+bwd kept-pair TFLOP/s", "unit": "TFLOP/s",
             "value": round(world * (ff + fb) / ((t_f + t_b) * 1e-3) / 1e12, 3),
             "config": {"workload": "train", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N, "d": wl.d, "w": wl.w,
@@ -415,6 +502,7 @@ def leg_train(args, world, torch, dma, peaks):
             "fwd_ms": round(t_f, 4), "bwd_ms": round(t_b, 4),
             "fwd_tflops": round(ff / (t_f * 1e-3) / 1e12, 2), "bwd_tflops": round(fb / (t_b * 1e-3) / 1e12, 2),
             "bwd_frac_of_peak": round(fb / (t_b * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "dense_causal": dense,
             "gpu_launches": 17 * n}   # forward 7, attention backward 6, gate backward 4
 
 

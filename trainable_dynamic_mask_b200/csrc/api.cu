@@ -53,9 +53,15 @@ cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
 
 // Work units of the attention forward (see FwdSchedule).  The split counts depend only on the
 // problem's shape and a fixed reference of 148 SMs, so that the workspace plan and the launch agree.
-// Splitting costs a second pipeline start and a merge per split pair, so pairs are split only when
-// there are fewer pairs than SMs: then each pair gets S = min(4, ceil(SMs / pairs), its tiles)
-// splits (its list length estimated as min(t1, min(w, N) + 128) keys).
+// A pair's list length is estimated as min(t1, min(w, N) + 128) keys.  The persistent CTAs take the
+// units heaviest first in snake order, so the kernel ends when the CTA with the most tiles does.
+// A unit of more than half the average tiles per SM ("big") cannot share a CTA with another big
+// one without pushing that CTA past the average: when there are more big units than SMs (e.g. 208
+// of ~9 tiles on 148 SMs for 16 heads x 16 pairs), whole groups of big pairs, heaviest first, are
+// split in two until the big units fit one per SM.  Each split costs a second pipeline start and a
+// merge of partial (O, m, l) by the split that finishes last (a few us), which is why pairs are not
+// split further.  When there are fewer pairs than SMs, each pair gets
+// min(kMaxSplits, ceil(SMs / pairs), tiles) units.
 void fwd_schedule(const Plan& P, FwdSchedule* S) {
   constexpr int kRefSMs = 148;
   const int BH = P.B * P.H;
@@ -63,14 +69,33 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
   const long items = (long)BH * P.n_pairs;
   const long want = items >= kRefSMs ? 1 : (kRefSMs + items - 1) / items;
   int est[kMaxPairs], split[kMaxPairs], order[kMaxPairs];
+  long total = 0;
   for (int kp = 0; kp < P.n_pairs; ++kp) {
     const int t1 = (kp + 1) * kPairQ < P.N ? (kp + 1) * kPairQ : P.N;
     const int live = t1 < minwn + kBlockQ ? t1 : minwn + kBlockQ;
     est[kp] = (live + kBlockQ - 1) / kBlockQ;
+    total += est[kp];
     long sp = want < kMaxSplits ? want : kMaxSplits;
     if (sp > est[kp]) sp = est[kp];
     split[kp] = (int)(sp < 1 ? 1 : sp);
     order[kp] = kp;
+  }
+  total *= BH;
+  if (want == 1) {
+    // big: 2 * est * SMs > total (more than half the average per SM)
+    auto is_big = [&](long tiles, long parts) { return 2 * tiles * kRefSMs > total * parts; };
+    long big = 0;
+    for (int kp = 0; kp < P.n_pairs; ++kp)
+      if (is_big(est[kp], 1)) big += BH;
+    while (big > kRefSMs) {
+      int pick = -1;
+      for (int kp = 0; kp < P.n_pairs; ++kp)
+        if (split[kp] == 1 && est[kp] >= 2 && is_big(est[kp], 1) && (pick < 0 || est[kp] >= est[pick])) pick = kp;
+      if (pick < 0) break;
+      split[pick] = 2;
+      big -= BH;
+      if (is_big(est[pick], 2)) big += 2L * BH;
+    }
   }
   // heaviest units first: cost est / S, ties to the later pair
   for (int a = 1; a < P.n_pairs; ++a)
