@@ -53,6 +53,7 @@ __all__ = [
     "attn_bwd",
     "gate_bwd",
     "decode_select",
+    "decode_select_append",
     "decode_attn",
 ]
 
@@ -348,6 +349,46 @@ def decode_select(delta: np.ndarray, w: int) -> np.ndarray:
             d = np.asarray(delta[b, h], dtype=np.float32).astype(np.float64)
             order = np.lexsort((idx, -d))       # primary -delta, secondary index
             out[b, h] = np.sort(order[:k])
+    return out
+
+
+def decode_select_append(prev_sel: np.ndarray, delta: np.ndarray, w: int) -> np.ndarray:
+    """The decode selection after one key is appended to the cache, from the
+    previous one (the "Unified Training-Inference Architecture" section: the
+    same selection at every decode step; the m_t equation: the query at
+    position t keeps the min(t+1, w) best keys of [0, t]).
+
+    Because delta_j does not depend on the query, the best keys of [0, t] are
+    the best of (the best keys of [0, t-1]) plus key t.  So with fewer than w
+    keys selected the new key joins; otherwise it replaces the worst selected
+    key (smallest delta; on equal delta the larger index, which loses the
+    lower-index-first rule) exactly when it is better under the selection
+    order.  The new key has the largest index, so that is when its delta is
+    strictly larger.
+
+    prev_sel [B, H, min(L-1, w)] ascending (the selection over the first L-1
+    keys); delta [B, H, L].  Returns [B, H, min(L, w)] ascending, int64.
+    """
+    B, H, L = delta.shape
+    kp = prev_sel.shape[2]
+    assert kp == min(L - 1, w)
+    k = min(L, w)
+    out = np.empty((B, H, k), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            d = np.asarray(delta[b, h], dtype=np.float32)
+            cur = [int(j) for j in prev_sel[b, h]]
+            if kp < w:
+                cur.append(L - 1)
+            else:
+                worst = cur[0]
+                for j in cur[1:]:
+                    if d[j] < d[worst] or (d[j] == d[worst] and j > worst):
+                        worst = j
+                if d[L - 1] > d[worst]:
+                    cur.remove(worst)
+                    cur.append(L - 1)
+            out[b, h] = cur
     return out
 
 

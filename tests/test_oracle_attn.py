@@ -242,6 +242,30 @@ def test_decode_select_is_last_row_of_the_selection():
                 np.testing.assert_array_equal(sel[b, h], np.nonzero(M[L - 1])[0])
 
 
+def test_decode_select_append_equals_the_full_selection_at_every_length():
+    # growing the cache key by key from one key, across the point where min(L, w) stops growing,
+    # on uniform, heavily tied and constant gate values (ties test the lower-index-first rule)
+    B, H, L, w = 2, 3, 90, 16
+    for kind in ("uniform", "levels", "constant"):
+        delta = make_delta((B, H, L), seed=33, kind=kind, levels=4)
+        sel = oracle.decode_select(delta[:, :, :1], w)
+        for n in range(2, L + 1):
+            sel = oracle.decode_select_append(sel, delta[:, :, :n], w)
+            np.testing.assert_array_equal(sel, oracle.decode_select(delta[:, :, :n], w), err_msg=f"{kind} L={n}")
+
+
+def test_decode_select_append_cases():
+    # hand-checked: w = 3, delta of keys 0..3 = [0.5, 0.2, 0.9, x]
+    d = np.array([[[0.5, 0.2, 0.9, 0.0]]], dtype=np.float32)
+    prev = np.array([[[0, 1, 2]]])
+    for x, want in ((0.1, [0, 1, 2]), (0.2, [0, 1, 2]), (0.3, [0, 2, 3]), (1.0, [0, 2, 3])):
+        d[0, 0, 3] = x
+        np.testing.assert_array_equal(oracle.decode_select_append(prev, d, 3)[0, 0], want, err_msg=str(x))
+    # equal worst values: the larger index is the worst (key 2 goes, not key 1)
+    d = np.array([[[0.9, 0.2, 0.2, 0.5]]], dtype=np.float32)
+    np.testing.assert_array_equal(oracle.decode_select_append(np.array([[[0, 1, 2]]]), d, 3)[0, 0], [0, 1, 3])
+
+
 def test_decode_attn_is_last_row_of_prefill():
     Q, K, V = _rand(13, B=2, H=4, Hkv=2, N=64, d=8)
     delta = make_delta(Q.shape[:3], seed=13).astype(np.float64)

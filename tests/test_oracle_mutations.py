@@ -3,7 +3,9 @@
 Each case plants one mistake in the oracle (on the CPU, through monkeypatch)
 and checks that at least one pin then fails: a dropped term of softplus, the
 tie rule reversed, the scale applied to delta as well, a transposed Delta, a
-missing row-max subtraction sign, a wrong sign in the backward.
+missing row-max subtraction sign, a wrong sign in the backward, and the two tie
+mistakes of the decode append rule (an equal new key entering; the smaller
+index leaving among equal worst keys).
 """
 import math
 
@@ -96,3 +98,38 @@ def test_wrong_sign_in_backward_is_caught(monkeypatch):
 def test_gate_backward_missing_sigmoid_is_caught(monkeypatch):
     monkeypatch.setattr(od, "sigmoid", lambda x: np.ones_like(np.asarray(x, dtype=np.float64)))
     assert _fails(TA.test_gate_backward_matches_central_differences)
+
+
+def _append_with(ge: bool, smaller_index_is_worst: bool):
+    def bad(prev_sel, delta, w):
+        B, H, L = delta.shape
+        out = []
+        for b in range(B):
+            rows = []
+            for h in range(H):
+                d = np.asarray(delta[b, h], dtype=np.float32)
+                cur = [int(j) for j in prev_sel[b, h]]
+                if len(cur) < w:
+                    cur.append(L - 1)
+                else:
+                    worst = cur[0]
+                    for j in cur[1:]:
+                        tie_pick = j < worst if smaller_index_is_worst else j > worst
+                        if d[j] < d[worst] or (d[j] == d[worst] and tie_pick):
+                            worst = j
+                    if (d[L - 1] >= d[worst]) if ge else (d[L - 1] > d[worst]):
+                        cur.remove(worst)
+                        cur.append(L - 1)
+                rows.append(sorted(cur))
+            out.append(rows)
+        return np.array(out, dtype=np.int64)
+    return bad
+
+
+@pytest.mark.parametrize("ge, smaller", [(True, False), (False, True)])
+def test_append_tie_mistakes_are_caught(monkeypatch, ge, smaller):
+    # a new key that only equals the worst one must not enter; among equal worst values the larger
+    # index leaves
+    monkeypatch.setattr(oracle, "decode_select_append", _append_with(ge, smaller))
+    assert _fails(TA.test_decode_select_append_equals_the_full_selection_at_every_length) or \
+        _fails(TA.test_decode_select_append_cases)
