@@ -393,6 +393,26 @@ def leg_decode(args, world, torch, dma, peaks):
     t_sel = _max_over_ranks(t_sel, world, torch) / n
     t_att = _max_over_ranks(t_att, world, torch) / n
     gbs = bytes_unique / (t_att * 1e-3) / 1e9
+    # the incremental selection: one key appended to a cache of L - 1 keys (the selection over L - 1
+    # keys is restored before every timed call; the result must equal the full selection)
+    sel_bytes = wl.B * wl.H * lay.sel_len * 4
+    full_sel = ws[lay.off_sel: lay.off_sel + sel_bytes].clone()
+    p_prev = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N - 1, wl.d, wl.w, Nq=1, dtype="bf16")
+    dma.topk_mask(p_prev, delta[:, :, :wl.N - 1].contiguous(), None, ws)
+    prev_sel = ws[lay.off_sel: lay.off_sel + sel_bytes].clone()
+    t_app = 0.0
+    for i in range(args.warmup + n):
+        ws[lay.off_sel: lay.off_sel + sel_bytes].copy_(prev_sel)
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dma.topk_append(p, delta, ws)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            t_app += a.elapsed_time(b)
+    t_app = _max_over_ranks(t_app, world, torch) / n
+    append_ok = bool(torch.equal(ws[lay.off_sel: lay.off_sel + sel_bytes], full_sel))
     # the same kernels with w = L (every cached row attended), timed the same way
     p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, Nq=1, dtype="bf16")
     ws_d = dma.alloc_workspace(p_d)
@@ -416,12 +436,13 @@ def leg_decode(args, world, torch, dma, peaks):
     return {"metric": "decode selected-KV GB/s", "value": round(world * gbs, 2), "unit": "GB/s",
             "config": {"workload": "decode", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "L": wl.N, "d": wl.d, "w": wl.w},
             "attn_us": round(t_att * 1e3, 2), "select_us": round(t_sel * 1e3, 2),
+            "select_append_us": round(t_app * 1e3, 2), "append_equals_full_selection": append_ok,
             "roofline": {"kernel": "decode_split+combine", "bound": "hbm", "achieved": round(gbs, 2),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "peak_kind": peaks["source"], "traffic": None,
                          "algorithmic_bytes": bytes_unique, "bytes_if_per_head": bytes_per_head},
             "dense_causal": dense,
-            "gpu_launches": 3 * n}
+            "gpu_launches": 4 * n}
 
 
 def leg_train(args, world, torch, dma, peaks):

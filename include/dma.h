@@ -165,6 +165,33 @@ dma_status_t dma_topk_mask(const dma_params_t* p, const float* delta, int32_t* e
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Decode selection after one key is appended to the cache (section "Unified Training-Inference
+ * Architecture": the same selection at every decode step).  p: decode parameters (Nq == 1) with
+ * N = L >= 2, the cache length including the new key at position L-1, whose gate value is in
+ * delta [B, H, L] float32.  Because delta_j does not depend on the query, the best keys of [0, L)
+ * are the best of those of [0, L-1) plus the new key: while fewer than w keys are selected it
+ * joins; otherwise it replaces the worst selected key (smallest delta, the larger index among
+ * equal ones) when its delta is strictly larger.  O(min(L, w)) work per (b, h) instead of a
+ * selection over all L keys.  Writes to the workspace region off_sel exactly what dma_topk_mask
+ * writes for N = L.  When L - 1 > w the region must already hold the selection over the first
+ * L - 1 keys (dma_topk_mask or dma_topk_append with N = L - 1 and the same B, H, w, on the same
+ * workspace); otherwise (every earlier key is selected) nothing is read from it.
+ */
+dma_status_t dma_topk_append(const dma_params_t* p, const float* delta, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * Gate of the last key position only (the key just appended to a decode cache), "Dynamic Weight
+ * Computation" equation: delta[b, h, N-1] = exp(A_h softplus(x)),
+ * x = sum_{g,c} V[b, g, N-1, c] Delta[g*d + c, h]; x_save[b, h, N-1] = x when x_save is not NULL.
+ * Other positions of delta and x_save are left as they are.  V [B, Hkv, N, d] dtype (the cache),
+ * Delta [Hkv*d, H] dtype, A [H] float32.  Within the gate's float32 tolerance of dma_gate (the sum
+ * runs in another order).  Needs no workspace.
+ */
+dma_status_t dma_gate_append(const dma_params_t* p, const void* V, const void* Delta, const float* A,
+                             float* delta, float* x_save, void* stream);
+
+/*
  * Masked attention forward (o_t equation), computing only on the live keys of each block
  * (masked pairs are skipped, section "Theoretical Guarantees for Safe Computation Skipping").
  *   Q      [B, H, Nq, d] dtype;  K, V [B, Hkv, N, d] dtype;  delta [B, H, N] float32

@@ -138,6 +138,13 @@ assert lib.dma_attn_bwd(pp, *args_bad) == INVALID
 assert lib.dma_gate_bwd(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
 # gate_bwd_noalloc(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, stream)
 assert lib.dma_gate_bwd_noalloc(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == INVALID
+# topk_append(p, delta, ws, ws_bytes, stream): decode parameters only, a workspace of the plan's size
+assert lib.dma_topk_append(pp, FAKE, FAKE, need, None) == INVALID
+assert lib.dma_topk_append(ctypes.byref(pd), None, FAKE, needd, None) == INVALID
+assert lib.dma_topk_append(ctypes.byref(pd), FAKE, FAKE, needd - 1, None) == WORKSPACE
+# gate_append(p, V, Delta, A, delta, x_save, stream)
+assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, None, None, None) == INVALID
+assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE + 4, None) == INVALID
 pdec = dma.make_params(8, 32, 8, 65536, 128, 2048, Nq=1)   # 64 MiB of gx alone: more than the fixed array
 assert lib.dma_gate_bwd_noalloc(ctypes.byref(pdec), *([FAKE] * 9), None) == UNSUPPORTED
 print("ok")

@@ -131,3 +131,53 @@ def test_decode_select(L, w, kind):
     lay = dma.workspace_layout(p)
     sel = ws.cpu().numpy()[lay.off_sel: lay.off_sel + B * H * lay.sel_len * 4].view(np.int32).reshape(B, H, -1)
     np.testing.assert_array_equal(sel, oracle.decode_select(d, w))
+
+
+# ---------------------------------------------------------------- decode: one key appended
+
+def _sel_of(dma, p, ws):
+    lay = dma.workspace_layout(p)
+    B, H = p.B, p.H
+    return ws.cpu().numpy()[lay.off_sel: lay.off_sel + B * H * lay.sel_len * 4].view(np.int32).reshape(B, H, -1)
+
+
+@pytest.mark.parametrize("L0,L,w,kind", [(2, 70, 16, "uniform"), (2, 70, 16, "levels"), (30, 200, 33, "constant"),
+                                         (3000, 3012, 2048, "levels"), (65535, 65536, 2048, "uniform")])
+def test_decode_select_append(L0, L, w, kind):
+    """dma_topk_append grows the selection key by key (from none while L <= w + 1, else from
+    dma_topk_mask at L0); after every key it equals the oracle's selection over the whole prefix."""
+    dma = lib()
+    torch = torch_cuda()
+    B, H = 2, 3
+    d = make_delta((B, H, L), seed=L0 + L + w, kind=kind, levels=6)
+    ws = torch.empty(dma.workspace_size(dma.make_params(B, H, H, L, 128, w, Nq=1)), dtype=torch.uint8, device="cuda")
+    if L0 - 1 > w:
+        p0 = dma.make_params(B, H, H, L0 - 1, 128, w, Nq=1)
+        dma.topk_mask(p0, f32_dev(d[:, :, :L0 - 1]), None, ws)
+    for n in range(L0, L + 1):
+        p = dma.make_params(B, H, H, n, 128, w, Nq=1)
+        dma.topk_append(p, f32_dev(d[:, :, :n]), ws)
+        torch.cuda.synchronize()
+        if n == L or n - L0 < 40 or n % 17 == 0:
+            np.testing.assert_array_equal(_sel_of(dma, p, ws), oracle.decode_select(d[:, :, :n], w), err_msg=f"L={n}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_gate_append(dtype):
+    """dma_gate_append writes delta (and x) at position N-1 only, within the gate's tolerance."""
+    dma = lib()
+    torch = torch_cuda()
+    wl = get("decode").with_(B=2, N=3000, dtype=dtype, seed=71)
+    I = make_inputs(wl)
+    p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, Nq=1, dtype=dtype)
+    V = to_dev(I.V, I.bits.get("V"), dtype)
+    D = to_dev(I.Delta, I.bits.get("Delta"), dtype)
+    delta = torch.full((wl.B, wl.H, wl.N), float("nan"), dtype=torch.float32, device="cuda")
+    x = torch.full_like(delta, float("nan"))
+    dma.gate_append(p, V, D, f32_dev(I.A), delta, x)
+    torch.cuda.synchronize()
+    x_ref, d_ref = oracle.gate(I.V, I.Delta, I.A)
+    got_d, got_x = to_np(delta), to_np(x)
+    assert_delta_close(got_d[:, :, -1:], d_ref[:, :, -1:])
+    np.testing.assert_allclose(got_x[:, :, -1], x_ref[:, :, -1], rtol=1e-5, atol=1e-5)
+    assert np.isnan(got_d[:, :, :-1]).all() and np.isnan(got_x[:, :, :-1]).all()

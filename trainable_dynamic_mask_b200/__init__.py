@@ -18,7 +18,8 @@ from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DmaError, DmaParams, DmaWsLayout,
 
 __all__ = [
     "BLOCK_Q", "DMA_BF16", "DMA_F32", "DmaError", "DmaParams", "LIB_PATH", "load", "exported_names",
-    "make_params", "workspace_size", "workspace_layout", "gate", "topk_mask", "attn_fwd", "attn_bwd",
+    "make_params", "workspace_size", "workspace_layout", "gate", "topk_mask", "topk_append", "gate_append",
+    "attn_fwd", "attn_bwd",
     "gate_bwd", "gate_bwd_noalloc", "check_device_status", "clear_device_status", "abi_version", "alloc_workspace", "forward",
     "backward",
 ]
@@ -80,6 +81,18 @@ def gate(p, V, Delta, A, delta, x_save=None, workspace=None, stream=None):
 def topk_mask(p, delta, evict, workspace, stream=None):
     check("dma_topk_mask", load().dma_topk_mask(ctypes.byref(p), _ptr(delta), _ptr(evict),
                                                 _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def topk_append(p, delta, workspace, stream=None):
+    """Decode selection after one key is appended (p.N = the new cache length)."""
+    check("dma_topk_append", load().dma_topk_append(ctypes.byref(p), _ptr(delta), _ptr(workspace),
+                                                    _nbytes(workspace), _stream(stream)))
+
+
+def gate_append(p, V, Delta, A, delta, x_save=None, stream=None):
+    """Gate of the last key position only (delta[:, :, p.N - 1])."""
+    check("dma_gate_append", load().dma_gate_append(ctypes.byref(p), _ptr(V), _ptr(Delta), _ptr(A), _ptr(delta),
+                                                    _ptr(x_save), _stream(stream)))
 
 
 def attn_fwd(p, Q, K, V, delta, evict, workspace, O, LSE, stream=None):

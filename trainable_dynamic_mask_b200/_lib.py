@@ -44,6 +44,8 @@ _SIGS = {
     "dma_workspace_layout": [ctypes.POINTER(DmaParams), ctypes.POINTER(DmaWsLayout)],
     "dma_gate": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp],
     "dma_topk_mask": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_sz, c_vp],
+    "dma_topk_append": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_sz, c_vp],
+    "dma_gate_append": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp],
     "dma_attn_fwd": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp,
                      c_vp],
     "dma_attn_bwd": [ctypes.POINTER(DmaParams), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp,

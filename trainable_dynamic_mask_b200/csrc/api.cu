@@ -283,6 +283,26 @@ dma_status_t dma_topk_mask(const dma_params_t* p, const float* delta, int32_t* e
   return cuda_status(launch_topw_prefill(P, delta, evict, workspace, s));
 }
 
+dma_status_t dma_topk_append(const dma_params_t* p, const float* delta, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!P.decode || !ok_ptr(delta)) return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  return cuda_status(launch_topw_append(P, delta, workspace, (cudaStream_t)stream));
+}
+
+dma_status_t dma_gate_append(const dma_params_t* p, const void* V, const void* Delta, const float* A,
+                             float* delta, float* x_save, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (!ok_ptr(V) || !ok_ptr(Delta) || !ok_ptr(A) || !ok_ptr(delta) || (x_save != nullptr && !ok_ptr(x_save)))
+    return DMA_ERR_INVALID_ARG;
+  return cuda_status(launch_gate_append(P, V, Delta, A, delta, x_save, (cudaStream_t)stream));
+}
+
 dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
                           const float* delta, const int32_t* evict, void* workspace,
                           size_t workspace_bytes, void* O, float* LSE, void* stream) {

@@ -478,6 +478,44 @@ cudaError_t launch_gate_fwd_h(const Plan& P, const void* V, const void* Delta, c
 
 }  // namespace
 
+// ---------------------------------------------------------------- gate of the last position
+// One warp per (b, h): x = sum_{g,c} V[b, g, N-1, c] Delta[g*d + c, h] in float32, then
+// delta = exp(A_h softplus(x)), at position N - 1 only.
+template <typename T>
+__global__ void gate_append_kernel(const T* __restrict__ V, const T* __restrict__ Delta, const float* __restrict__ A,
+                                   float* __restrict__ delta, float* __restrict__ x_save, int BH, int H, int Hkv,
+                                   int N, int d) {
+  const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+  if (gw >= BH) return;
+  const int b = gw / H, h = gw % H;
+  float acc = 0.f;
+  for (int r = lane; r < Hkv * d; r += 32) {
+    const int g = r / d, c = r % d;
+    acc = fmaf(load_as_f32(V + ((size_t)(b * Hkv + g) * N + (N - 1)) * d + c), load_as_f32(Delta + (size_t)r * H + h),
+               acc);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    const size_t off = (size_t)gw * N + (N - 1);
+    delta[off] = expf(A[h] * softplus_f(acc));
+    if (x_save) x_save[off] = acc;
+  }
+}
+
+cudaError_t launch_gate_append(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
+                               float* x_save, cudaStream_t s) {
+  const int BH = P.B * P.H;
+  const unsigned blocks = (unsigned)((BH * 32 + 255) / 256);
+  if (P.bf16)
+    gate_append_kernel<uint16_t><<<blocks, 256, 0, s>>>((const uint16_t*)V, (const uint16_t*)Delta, A, delta, x_save,
+                                                        BH, P.H, P.Hkv, P.N, P.d);
+  else
+    gate_append_kernel<float><<<blocks, 256, 0, s>>>((const float*)V, (const float*)Delta, A, delta, x_save, BH, P.H,
+                                                     P.Hkv, P.N, P.d);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, const float* A,
                             float* delta, float* x_save, cudaStream_t s) {
   if (gate_mma_smem(P) > 0) {

@@ -809,6 +809,69 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- decode: one key appended
+constexpr int kAppThreads = 256;
+
+// One CTA per (b, h) row: the selection over [0, L) from the one over [0, L-1) (stride w when
+// L - 1 > w; every key when L - 1 <= w, then not read).  The worst selected key is the smallest
+// (order key, ~index) composite: the smallest delta, the larger index among equal ones.  The new
+// key L - 1 enters iff its order key is strictly larger; it then has the largest index, so the
+// ascending list loses the worst key's entry and gains L - 1 at its end.
+__global__ void __launch_bounds__(kAppThreads)
+topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int L, int w) {
+  __shared__ uint64_t wmin[kAppThreads / 32];
+  __shared__ int pos;
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* drow = delta + (size_t)row * L;
+  const int kp = min(L - 1, w), k = min(L, w);
+  int32_t* out = sel + (size_t)row * k;
+  if (kp < w) {   // every key is selected
+    for (int i = tid; i < L; i += kAppThreads) out[i] = i;
+    return;
+  }
+  const bool implicit = L - 1 == w;   // the previous selection is every key 0 .. L-2
+  uint64_t c = ~0ull;
+  for (int i = tid; i < w; i += kAppThreads) {
+    const int j = implicit ? i : out[i];
+    c = min(c, ((uint64_t)order_key(drow[j]) << 32) | (uint64_t)(~(uint32_t)j));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c = min(c, __shfl_xor_sync(0xffffffffu, c, o));
+  if (lane == 0) wmin[warp] = c;
+  if (tid == 0) pos = w;
+  __syncthreads();
+  c = wmin[0];
+#pragma unroll
+  for (int i = 1; i < kAppThreads / 32; ++i) c = min(c, wmin[i]);
+  const uint32_t okw = (uint32_t)(c >> 32);
+  const int jw = (int)~(uint32_t)c;
+  const bool enter = order_key(drow[L - 1]) > okw;
+  if (implicit) {
+    for (int i = tid; i < w; i += kAppThreads) out[i] = (!enter || i < jw) ? i : i + 1;
+    return;
+  }
+  if (!enter) return;
+  for (int i = tid; i < w; i += kAppThreads)
+    if (out[i] == jw) pos = i;   // the keys are distinct: one writer
+  __syncthreads();
+  const int p0 = pos;
+  // entries [p0, w - 1) move down by one, then L - 1 at the end; rounds in ascending order read
+  // every entry before it is overwritten
+  for (int base = (p0 / kAppThreads) * kAppThreads; base < w; base += kAppThreads) {
+    const int i = base + tid;
+    int v = 0;
+    if (i >= p0 && i < w) v = i + 1 < w ? out[i + 1] : L - 1;
+    __syncthreads();
+    if (i >= p0 && i < w) out[i] = v;
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
+  topw_append_kernel<<<P.B * P.H, kAppThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
   const int smem = (int)sizeof(SelShared);
   { cudaError_t ea = ensure_smem_limit(topw_decode_kernel, smem); if (ea != cudaSuccess) return ea; }
