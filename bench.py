@@ -151,9 +151,12 @@ def _to_dev_bf16(bits, torch):
 
 
 def _max_over_ranks(x: float, world: int, torch) -> float:
+    """The maximum of x over the ranks (the device timings of a step are reported as the slowest
+    rank's).  The reduction runs on the process group's device: CUDA for NCCL, the host for gloo."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -161,7 +164,8 @@ def _max_over_ranks(x: float, world: int, torch) -> float:
 def _barrier(world, torch):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 # ---------------------------------------------------------------- our arm
