@@ -203,8 +203,9 @@ def live_keys_per_block(e: np.ndarray, Bq: int):
 # Masked attention forward / backward
 # ----------------------------------------------------------------------------
 
-def _scores(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype):
-    """Scaled scores plus the additive mask of rows `rows`.
+def _scores(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype, q_pos0=0):
+    """Scaled scores plus the additive mask of rows `rows` (query row i sits
+    at position q_pos0 + i).
 
     Reading of the garbled operator in the o_t equation: the mask m_t is added
     to q_t k^T / sqrt(d): selected key j contributes +delta_j, non-selected
@@ -213,7 +214,7 @@ def _scores(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype):
     s = np.matmul(np.asarray(Qh[rows], dtype=gemm_dtype),
                   np.asarray(Kg, dtype=gemm_dtype).T).astype(np.float64) * scale
     s = s + np.asarray(delta_h, dtype=np.float64)[None, :]
-    t = np.asarray(rows)[:, None] if rows is not None else np.arange(Qh.shape[0])[:, None]
+    t = q_pos0 + (np.asarray(rows)[:, None] if rows is not None else np.arange(Qh.shape[0])[:, None])
     j = np.arange(N)[None, :]
     sel = (j <= t) & (t < np.asarray(e_h)[None, :])
     return np.where(sel, s, -np.inf), sel
@@ -230,10 +231,10 @@ def attn_fwd(Q, K, V, delta, evict, scale=None, q_pos0: int = 0, rows=None,
     a subset of query rows (other rows are NaN).
 
     Dense definition: every causal key is scored, non-selected ones get -inf,
-    softmax with max subtraction, O = P V.
+    softmax with max subtraction, O = P V.  With q_pos0 > 0 the queries are a
+    chunk of a longer sequence (positions q_pos0 .. q_pos0 + Nq - 1) over all
+    N keys, with the selection of the whole sequence.
     """
-    if q_pos0 != 0:
-        raise NotImplementedError("query rows at an offset: use decode_attn")
     B, H, Nq, d = Q.shape
     Hkv, N = K.shape[1], K.shape[2]
     G = H // Hkv
@@ -247,7 +248,7 @@ def attn_fwd(Q, K, V, delta, evict, scale=None, q_pos0: int = 0, rows=None,
             g = h // G
             for c0 in range(0, all_rows.size, chunk):
                 r = all_rows[c0:c0 + chunk]
-                s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], r, scale, gemm_dtype)
+                s, _ = _scores(Q[b, h], K[b, g], delta[b, h], evict[b, h], r, scale, gemm_dtype, q_pos0)
                 m = s.max(axis=1, keepdims=True)
                 p = np.exp(s - m)
                 l = p.sum(axis=1, keepdims=True)

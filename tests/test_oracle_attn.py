@@ -266,6 +266,20 @@ def test_decode_select_append_cases():
     np.testing.assert_array_equal(oracle.decode_select_append(np.array([[[0, 1, 2]]]), d, 3)[0, 0], [0, 1, 3])
 
 
+def test_chunked_queries_are_rows_of_the_full_sequence():
+    # a chunk of queries at an offset sees the same keys and selection as those rows of the whole
+    # sequence; the last row also equals decode
+    Q, K, V = _rand(17, B=1, H=4, Hkv=2, N=90, d=8)
+    delta = make_delta(Q.shape[:3], seed=17).astype(np.float64)
+    w = 12
+    e = _evict(delta, w)
+    O, LSE = oracle.attn_fwd(Q, K, V, delta, e)
+    for q0 in (1, 37, 89):
+        Oc, Lc = oracle.attn_fwd(Q[:, :, q0:], K, V, delta, e, q_pos0=q0)
+        np.testing.assert_allclose(Oc, O[:, :, q0:], rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(Lc, LSE[:, :, q0:], rtol=1e-14)
+
+
 def test_decode_attn_is_last_row_of_prefill():
     Q, K, V = _rand(13, B=2, H=4, Hkv=2, N=64, d=8)
     delta = make_delta(Q.shape[:3], seed=13).astype(np.float64)
