@@ -341,7 +341,7 @@ def run_ours(args, world, rank):
     }
     legs = [] if args.no_legs else [x for x in args.legs.split(",") if x]
     if legs:
-        run = {"decode": leg_decode, "train": leg_train}
+        run = {"decode": leg_decode, "train": leg_train, "chunk": leg_chunk}
         line["legs"] = {name: run[name](args, world, torch, dma, peaks) for name in legs}
         line["gpu_launches"] += sum(leg["gpu_launches"] for leg in line["legs"].values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -447,6 +447,55 @@ def leg_decode(args, world, torch, dma, peaks):
                          "algorithmic_bytes": bytes_unique, "bytes_if_per_head": bytes_per_head},
             "dense_causal": dense,
             "gpu_launches": 4 * n}
+
+
+def leg_chunk(args, world, torch, dma, peaks):
+    """Chunked prefill: the last 2048 query positions of a 16384-key sequence (the long workload's
+    heads, window and seed), with the selection over all keys; kept-pair TFLOP/s of the attention."""
+    import numpy as np
+
+    from workloads import get, make_inputs
+    wl = get("long").with_(Nq=2048)
+    I = make_inputs(wl)
+    p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, Nq=wl.Nq, dtype="bf16")
+    Q, K, V = (_to_dev_bf16(I.bits[n], torch) for n in ("Q", "K", "V"))
+    Dl = _to_dev_bf16(I.bits["Delta"], torch)
+    A = torch.from_numpy(I.A).cuda()
+    del I
+    ws = dma.alloc_workspace(p)
+    delta = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device="cuda")
+    evict = torch.empty((wl.B, wl.H, wl.N), dtype=torch.int32, device="cuda")
+    O = torch.empty((wl.B, wl.H, wl.Nq, wl.d), dtype=torch.bfloat16, device="cuda")
+    LSE = torch.empty((wl.B, wl.H, wl.Nq), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    q0 = wl.N - wl.Nq
+    pairs = wl.B * wl.H * sum(min(t + 1, wl.w) for t in range(q0, wl.N))
+    flops = 4.0 * wl.d * pairs
+    n = max(5, min(args.steps // 10, 50))
+    t_step = t_att = 0.0
+    for i in range(args.warmup + n):
+        flush.zero_()
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record()
+        dma.gate(p, V, Dl, A, delta)
+        dma.topk_mask(p, delta, evict, ws)
+        b.record()
+        dma.attn_fwd(p, Q, K, V, delta, evict, ws, O, LSE)
+        c.record()
+        c.synchronize()
+        if i >= args.warmup:
+            t_step += a.elapsed_time(c)
+            t_att += b.elapsed_time(c)
+    t_step = _max_over_ranks(t_step, world, torch) / n
+    t_att = _max_over_ranks(t_att, world, torch) / n
+    tf = flops / (t_att * 1e-3) / 1e12
+    return {"metric": "chunked prefill attention kept-pair TFLOP/s", "value": round(world * tf, 2), "unit": "TFLOP/s",
+            "config": {"workload": "long with a chunk of queries", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N,
+                       "Nq": wl.Nq, "q0": q0, "d": wl.d, "w": wl.w, "kept_pairs": pairs},
+            "attn_us": round(t_att * 1e3, 2), "step_us": round(t_step * 1e3, 2),
+            "roofline": {"kernel": "attn_fwd", "bound": "tensor", "achieved": round(tf, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4)},
+            "gpu_launches": 7 * n}   # gate, top-w 5, attention
 
 
 def leg_train(args, world, torch, dma, peaks):
@@ -634,7 +683,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-legs", action="store_true", help="skip the decode and training legs")
-    ap.add_argument("--legs", default="decode,train", help="comma-separated legs to run: decode, train")
+    ap.add_argument("--legs", default="decode,train,chunk", help="comma-separated legs to run: decode, train, chunk")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)

@@ -78,8 +78,11 @@ typedef enum {
  *   H      query heads;  Hkv key/value heads, H % Hkv == 0 (grouped-query attention:
  *          query head h reads key/value head h / (H / Hkv))
  *   N      key length (sequence length, or cache length for decode)
- *   Nq     query rows: Nq == N (prefill / training; query row i sits at position i) or
- *          Nq == 1 (decode; the single query sits at position N-1)
+ *   Nq     query rows, 1 <= Nq <= N; the queries are the last Nq positions, query row i at
+ *          position N - Nq + i: Nq == N (prefill / training), Nq == 1 (decode), otherwise a
+ *          chunk of queries over a longer cache (chunked prefill: the selection still runs over
+ *          all N keys; the block lists and the attention cover the blocks from position N - Nq
+ *          on; dma_attn_bwd needs Nq == N)
  *   d      head dimension, 64 or 128
  *   w      window of the top-w selection, w >= 1 (w >= N keeps every causal key)
  *   scale  multiplier of q k^T; a value <= 0 selects 1/sqrt(d)
@@ -102,7 +105,8 @@ typedef struct {
  *   off_status  int32 device status word (0 = ok): kernels OR an error code into it (a bounded
  *               wait that gave up, an internal consistency check that failed).  Its content in a
  *               new workspace is undefined: clear it once with dma_clear_device_status.
- *   off_counts  int32 [B, H, n_blocks, 2]: per query block, (n_full, n_live).
+ *   off_counts  int32 [B, H, n_blocks, 2]: per query block, (n_full, n_live) (with Nq < N only
+ *               the blocks of pairs of blocks that hold a query row are written).
  *   off_lists   int32 [B, H, n_blocks, list_cap]: the live keys of each query block
  *               [t0, t1), t1 = min(t0 + DMA_BLOCK_Q, N): first the n_full "full" keys, selected
  *               by every row of the block (j <= t0 and e_j >= t1), then the partial ones (at

@@ -63,7 +63,8 @@ def _ws_size(p):
     (dict(B=1, H=2, Hkv=1, N=16385, d=64, w=4), UNSUPPORTED),   # prefill row limit
     (dict(B=1, H=2, Hkv=1, N=16384, d=128, w=4), OK),
     (dict(B=1, H=2, Hkv=1, N=65536, d=128, w=4, Nq=1), OK),     # decode has no such limit
-    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=4, Nq=7), INVALID),   # Nq must be N or 1
+    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=4, Nq=7), OK),        # a chunk of 7 queries at positions 249..255
+    (dict(B=1, H=2, Hkv=1, N=256, d=64, w=4, Nq=257), INVALID), # more queries than keys
     (dict(B=300, H=256, Hkv=1, N=256, d=64, w=4), UNSUPPORTED), # grid limit on B*H
 ])
 def test_params_validation(kw, expect):
@@ -138,6 +139,9 @@ assert lib.dma_attn_bwd(pp, *args_bad) == INVALID
 assert lib.dma_gate_bwd(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
 # gate_bwd_noalloc(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, stream)
 assert lib.dma_gate_bwd_noalloc(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == INVALID
+pc = dma.make_params(1, 2, 1, 256, 64, 64, Nq=100)   # chunked prefill: no backward
+args = [FAKE] * 6 + [need_of(pc)] + [FAKE] * 7 + [None]
+assert lib.dma_attn_bwd(ctypes.byref(pc), *args) == UNSUPPORTED
 # topk_append(p, delta, ws, ws_bytes, stream): decode parameters only, a workspace of the plan's size
 assert lib.dma_topk_append(pp, FAKE, FAKE, need, None) == INVALID
 assert lib.dma_topk_append(ctypes.byref(pd), None, FAKE, needd, None) == INVALID

@@ -35,7 +35,7 @@ def _setup(wl, with_dO=False, bf16_values=False):
     if with_dO:
         dev["dO"] = to_dev(I.dO, I.bits.get("dO"), wl.dtype)
     e_ref = None
-    if wl.Nq == wl.N:
+    if not (wl.Nq == 1 and wl.N > 1):   # prefill, training or a chunk of queries: eviction indices
         e_ref = np.stack([np.stack([oracle.topw_eviction(d32[b, h], wl.w) for h in range(wl.H)])
                           for b in range(wl.B)])
         dev["evict"] = torch.empty((wl.B, wl.H, wl.N), dtype=torch.int32, device="cuda")
@@ -66,6 +66,26 @@ FWD_CASES = {
     "n300_w1": get("tiny").with_(B=1, H=2, Hkv=1, N=300, d=128, w=1, dtype="f32", seed=24),
     "mha_n1000_w200": get("tiny").with_(B=2, H=3, Hkv=3, N=1000, d=128, w=200, dtype="bf16", seed=25),
 }
+
+
+CHUNK_CASES = {   # the queries are the last Nq positions of the N keys (chunked prefill)
+    "n3000_q700_w500": get("tiny").with_(B=1, H=4, Hkv=2, N=3000, Nq=700, d=128, w=500, dtype="bf16", seed=61),
+    "n4096_q1000_w1024": get("prefill").with_(H=4, Hkv=2, N=4096, Nq=1000, seed=62),
+    "n2048_q256_w300_d64": get("tiny").with_(B=2, H=2, Hkv=1, N=2048, Nq=256, d=64, w=300, dtype="bf16", seed=63),
+    "n1500_q1499_w200": get("tiny").with_(B=1, H=2, Hkv=2, N=1500, Nq=1499, d=128, w=200, dtype="bf16", seed=64),
+    "n700_q3_w_ge_n": get("tiny").with_(B=1, H=2, Hkv=1, N=700, Nq=3, d=128, w=900, dtype="f32", seed=65),
+}
+
+
+@pytest.mark.parametrize("case", list(CHUNK_CASES))
+def test_attn_fwd_chunked(case):
+    wl = CHUNK_CASES[case]
+    dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl)
+    O, LSE = _fwd(dma, torch, wl, p, ws, dev)
+    O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, q_pos0=wl.N - wl.Nq,
+                                   gemm_dtype=np.float32 if wl.N > 1024 else np.float64)
+    assert_close(to_np(LSE), L_ref, "LSE")
+    assert_close(to_np(O), O_ref, "O")
 
 
 @pytest.mark.parametrize("case", list(FWD_CASES))

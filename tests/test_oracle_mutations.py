@@ -66,8 +66,8 @@ def test_reversed_tie_rule_is_caught(monkeypatch):
 def test_scaling_delta_too_is_caught(monkeypatch):
     real = od._scores
 
-    def bad(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype):
-        return real(Qh, Kg, np.asarray(delta_h) * scale, e_h, rows, scale, gemm_dtype)
+    def bad(Qh, Kg, delta_h, e_h, rows, scale, gemm_dtype, q_pos0=0):
+        return real(Qh, Kg, np.asarray(delta_h) * scale, e_h, rows, scale, gemm_dtype, q_pos0)
 
     monkeypatch.setattr(od, "_scores", bad)
     assert _fails(TA.test_full_window_is_dense_causal_attention_with_bias)

@@ -66,11 +66,13 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
   constexpr int kRefSMs = 148;
   const int BH = P.B * P.H;
   const int minwn = P.w < P.N ? P.w : P.N;
-  const long items = (long)BH * P.n_pairs;
+  const int kp0 = P.q0 / kPairQ;        // pairs below the first query row have no query (chunked prefill)
+  const int np = P.n_pairs - kp0;
+  const long items = (long)BH * np;
   const long want = items >= kRefSMs ? 1 : (kRefSMs + items - 1) / items;
   int est[kMaxPairs], split[kMaxPairs], order[kMaxPairs];
   long total = 0;
-  for (int kp = 0; kp < P.n_pairs; ++kp) {
+  for (int kp = kp0; kp < P.n_pairs; ++kp) {
     const int t1 = (kp + 1) * kPairQ < P.N ? (kp + 1) * kPairQ : P.N;
     const int live = t1 < minwn + kBlockQ ? t1 : minwn + kBlockQ;
     est[kp] = (live + kBlockQ - 1) / kBlockQ;
@@ -78,18 +80,18 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
     long sp = want < kMaxSplits ? want : kMaxSplits;
     if (sp > est[kp]) sp = est[kp];
     split[kp] = (int)(sp < 1 ? 1 : sp);
-    order[kp] = kp;
+    order[kp - kp0] = kp;
   }
   total *= BH;
   if (want == 1) {
     // big: 2 * est * SMs > total (more than half the average per SM)
     auto is_big = [&](long tiles, long parts) { return 2 * tiles * kRefSMs > total * parts; };
     long big = 0;
-    for (int kp = 0; kp < P.n_pairs; ++kp)
+    for (int kp = kp0; kp < P.n_pairs; ++kp)
       if (is_big(est[kp], 1)) big += BH;
     while (big > kRefSMs) {
       int pick = -1;
-      for (int kp = 0; kp < P.n_pairs; ++kp)
+      for (int kp = kp0; kp < P.n_pairs; ++kp)
         if (split[kp] == 1 && est[kp] >= 2 && is_big(est[kp], 1) && (pick < 0 || est[kp] >= est[pick])) pick = kp;
       if (pick < 0) break;
       split[pick] = 2;
@@ -98,7 +100,7 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
     }
   }
   // heaviest units first: cost est / S, ties to the later pair
-  for (int a = 1; a < P.n_pairs; ++a)
+  for (int a = 1; a < np; ++a)
     for (int b = a; b > 0; --b) {
       const int x = order[b - 1], y = order[b];
       if ((long)est[y] * split[x] > (long)est[x] * split[y] ||
@@ -111,7 +113,7 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
     }
   memset(S, 0, sizeof(*S));
   int start = 0, slot = 0;
-  for (int i = 0; i < P.n_pairs; ++i) {
+  for (int i = 0; i < np; ++i) {
     const int kp = order[i];
     S->g[i].kp = kp;
     S->g[i].S = split[kp];
@@ -120,7 +122,7 @@ void fwd_schedule(const Plan& P, FwdSchedule* S) {
     start += BH * split[kp];
     if (split[kp] > 1) slot += BH * split[kp];
   }
-  S->n_groups = P.n_pairs;
+  S->n_groups = np;
   S->n_units = start;
   S->n_slots = slot;
 }
@@ -131,7 +133,7 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     return DMA_ERR_INVALID_ARG;
   if (p->H % p->Hkv != 0) return DMA_ERR_INVALID_ARG;
   if (p->dtype != DMA_BF16 && p->dtype != DMA_F32) return DMA_ERR_INVALID_ARG;
-  if (p->Nq != p->N && p->Nq != 1) return DMA_ERR_INVALID_ARG;
+  if (p->Nq > p->N) return DMA_ERR_INVALID_ARG;
   if (!(p->scale == p->scale) || isinf(p->scale)) return DMA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return DMA_ERR_UNSUPPORTED;
   if ((int64_t)p->B * p->H > 65535) return DMA_ERR_UNSUPPORTED;
@@ -142,6 +144,7 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   R.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
   R.bf16 = p->dtype == DMA_BF16;
   R.decode = (p->Nq == 1 && p->N > 1);
+  R.q0 = p->N - p->Nq;
   if (!R.decode && p->N > kTopwMaxN) return DMA_ERR_UNSUPPORTED;
   if (R.decode && p->N > (1 << 24)) return DMA_ERR_UNSUPPORTED;
 
@@ -339,7 +342,7 @@ dma_status_t dma_attn_bwd(const dma_params_t* p, const void* Q, const void* K, c
   Plan P;
   dma_status_t st = make_plan(p, &P);
   if (st != DMA_OK) return st;
-  if (P.decode) return DMA_ERR_UNSUPPORTED;
+  if (P.decode || P.q0 != 0) return DMA_ERR_UNSUPPORTED;   // training: every position is a query
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(delta) || !ok_ptr(evict) || !ok_ptr(O) ||
       !ok_ptr(LSE) || !ok_ptr(dO) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !ok_ptr(d_delta))
     return DMA_ERR_INVALID_ARG;

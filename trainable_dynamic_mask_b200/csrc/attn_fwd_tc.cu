@@ -159,8 +159,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
                    const int32_t* __restrict__ plen, const float* __restrict__ pdl, OutT* __restrict__ O,
                    float* __restrict__ LSE, float* __restrict__ fpart, float* __restrict__ fml,
                    int32_t* __restrict__ fcnt, int32_t* __restrict__ status, int H, int G, int N, int n_pairs,
-                   int pair_cap, float scale_log2) {
+                   int pair_cap, float scale_log2, int q0) {
   using S = TcSmem<D>;
+  const int Nq = N - q0;   // the queries are positions [q0, N) (q0 > 0: a chunk of a longer sequence)
   extern __shared__ __align__(1024) unsigned char sm[];
   TcBars& bar = *reinterpret_cast<TcBars*>(sm + S::kBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -248,7 +249,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             for (int qh = 0; qh < 2; ++qh) {
               int rr[4];
 #pragma unroll
-              for (int u = 0; u < 4; ++u) rr[u] = it.bh * N + min(t0 + qh * 128 + 4 * grp + u, N - 1);
+              for (int u = 0; u < 4; ++u) rr[u] = it.bh * Nq + min(max(t0 + qh * 128 + 4 * grp + u - q0, 0), Nq - 1);
 #pragma unroll
               for (int hf = 0; hf < D / 64; ++hf)
                 tma_gather4(smem_u32(sm + S::kQ + qh * S::kTile) + hf * 16384 + goff, &qmap, hf * 64, rr[0], rr[1],
@@ -510,8 +511,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
         tc::fence_after();
       }
-      const bool valid = t < N;
-      OutT* orow = O + ((size_t)it.bh * N + (valid ? t : 0)) * D;
+      const bool valid = t >= q0 && t < N;   // a query row (rows of the first pair below q0 are not)
+      OutT* orow = O + ((size_t)it.bh * Nq + (valid ? t - q0 : 0)) * D;
       if (it.S == 1) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
@@ -524,7 +525,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           for (int u2 = 0; u2 < 32; ++u2) of[u2] = __uint_as_float(ov[u2]) * inv;
           if (valid) store_row32(orow + c * 32, of);
         }
-        if (valid) LSE[(size_t)it.bh * N + t] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
+        if (valid) LSE[(size_t)it.bh * Nq + t - q0] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
       } else {
         // Split pair: every split but the last to finish leaves (O unnormalised, m, l) in its slot;
         // the last one merges them with its own.  Counters per (pair, half): [arrivals, written].
@@ -599,7 +600,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             for (int u2 = 0; u2 < 32; ++u2) of[u2] *= inv;
             if (valid) store_row32(orow + c * 32, of);
           }
-          if (valid) LSE[(size_t)it.bh * N + t] = (Mb + __log2f(L)) * kLn2;
+          if (valid) LSE[(size_t)it.bh * Nq + t - q0] = (Mb + __log2f(L)) * kLn2;
           group_sync(h);
           if (r == 0) {   // leave the counters at zero for the next launch on the same mask
             mc[0] = 0;
@@ -622,7 +623,7 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
                         const float* delta, const int32_t* evict, void* ws, void* O, float* LSE,
                         cudaStream_t s) {
   CUtensorMap qm, km, vm;
-  if (!make_row_map(&qm, Q, (uint64_t)P.B * P.H * P.N, D) || !make_row_map(&km, K, (uint64_t)P.B * P.Hkv * P.N, D) ||
+  if (!make_row_map(&qm, Q, (uint64_t)P.B * P.H * P.Nq, D) || !make_row_map(&km, K, (uint64_t)P.B * P.Hkv * P.N, D) ||
       !make_row_map(&vm, V, (uint64_t)P.B * P.Hkv * P.N, D))
     return cudaErrorInvalidValue;
   auto k = attn_fwd_tc_kernel<D, OutT>;
@@ -639,7 +640,7 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
                                    ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE, ws_ptr<float>(ws, P.off_fpart),
                                    ws_ptr<float>(ws, P.off_fml), ws_ptr<int32_t>(ws, P.off_fcnt),
                                    ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_pairs, P.pair_cap,
-                                   P.scale * kLog2e);
+                                   P.scale * kLog2e, P.q0);
   return cudaGetLastError();
 }
 

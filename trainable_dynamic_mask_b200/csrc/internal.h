@@ -41,6 +41,8 @@ struct Plan {
   float scale;
   bool bf16;      // storage dtype is bf16 (else f32)
   bool decode;    // Nq == 1 and N > 1 ... the single query sits at position N-1
+  int q0;         // first query position, N - Nq: 0 (prefill), N - 1 (decode), else a chunk of a longer
+                  // sequence (chunked prefill: the queries are the last Nq positions)
   int n_blocks;   // query blocks of kBlockQ rows (prefill)
   int list_cap;   // entries per block list
   int n_pairs;    // query blocks of kPairQ rows (attention forward work items)

@@ -362,11 +362,11 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
                   int32_t* __restrict__ counts, int32_t* __restrict__ lists,
                   int32_t* __restrict__ pcounts, int32_t* __restrict__ plists,
                   int32_t* __restrict__ plen, float* __restrict__ pdl, int32_t* __restrict__ fcnt, int N,
-                  int list_cap, int pair_cap, int n_blocks, int n_pairs) {
+                  int list_cap, int pair_cap, int n_blocks, int n_pairs, int kp0) {
   // partial keys: block a (<= 2C), block b (<= 2C), pair (<= 4C)
   __shared__ int32_t part[8 * kC];
   __shared__ int32_t wsum[6][kListWarps];   // per warp: full count of list 0..2, partial count of 0..2
-  const int kp = blockIdx.x, row = blockIdx.y;
+  const int kp = kp0 + (int)blockIdx.x, row = blockIdx.y;   // pairs from kp0: the ones holding a query
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = kp * kPairQ;
   const bool has_b = t0 + kC < N;
@@ -801,11 +801,12 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w);
   topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
-  topw_lists_kernel<<<dim3(P.n_pairs, rows), kListThreads, 0, s>>>(
+  const int kp0 = P.q0 / kPairQ;
+  topw_lists_kernel<<<dim3(P.n_pairs - kp0, rows), kListThreads, 0, s>>>(
       evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
       ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
       ws_ptr<float>(ws, P.off_pdl), ws_ptr<int32_t>(ws, P.off_fcnt), P.N, P.list_cap, P.pair_cap, P.n_blocks,
-      P.n_pairs);
+      P.n_pairs, kp0);
   return cudaGetLastError();
 }
 
