@@ -54,7 +54,8 @@ cudaError_t ensure_smem_limit_impl(const void* kernel, int bytes) {
 // Work units of the attention forward (see FwdSchedule).  The split counts depend only on the
 // problem's shape and a fixed reference of 148 SMs, so that the workspace plan and the launch agree.
 // A pair's list length is estimated as min(t1, min(w, N) + 128) keys.  The persistent CTAs take the
-// units heaviest first in snake order, so the kernel ends when the CTA with the most tiles does.
+// units heaviest first as they finish earlier ones, so the kernel ends when the CTA with the most
+// tiles does.
 // A unit of more than half the average tiles per SM ("big") cannot share a CTA with another big
 // one without pushing that CTA past the average: when there are more big units than SMs (e.g. 208
 // of ~9 tiles on 148 SMs for 16 heads x 16 pairs), whole groups of big pairs, heaviest first, are
@@ -183,7 +184,7 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     fwd_schedule(R, &R.sched);
     R.off_fpart = take((size_t)R.sched.n_slots * 2 * R.d * kBlockQ * sizeof(float));
     R.off_fml = take((size_t)R.sched.n_slots * 2 * 2 * kBlockQ * sizeof(float));
-    R.off_fcnt = take(BH * R.n_pairs * 4 * sizeof(int32_t));
+    R.off_fcnt = take((BH * R.n_pairs * 4 + 2) * sizeof(int32_t));   // + the forward's unit counters
     R.off_rowD = take(BH * R.Nq * sizeof(float));
     {
       const size_t n_slots = BH * ((R.N + 1023) / 1024) * 8;   // windows of 1024 keys, tiles of 128

@@ -8,8 +8,9 @@
 // Work item = (b, h, pair of query blocks: 256 rows), walking the pair's live-key list (the union
 // of the two blocks' lists; full keys first) in tiles of 128 keys.  Each gathered K/V tile feeds
 // both 128-row halves, so the gather traffic per tensor-core FLOP is half that of 128-row items.
-// The kernel is persistent: one CTA per SM walks work units heaviest-first (snake order over the
-// CTAs), and the next unit's Q and first tiles load while the current one finishes.  A unit is a
+// The kernel is persistent: one CTA per SM takes work units, heaviest first, from a global counter
+// as it finishes earlier ones (greedy longest-first, balanced by the units' actual durations), and
+// the next unit's Q and first tiles load while the current one finishes.  A unit is a
 // pair, or one of S splits of a long pair's list: the split that finishes last merges the others'
 // partial (O, m, l) with its own, so that few heavy pairs still spread evenly over the SMs.
 //
@@ -52,10 +53,13 @@ constexpr int kTcBK = 128;                  // keys per tile
 constexpr int kKStages = 2, kVStages = 2;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr int kPolyEvery = 4;               // one pair in kPolyEvery takes the polynomial exp2
+constexpr int kSchedRing = 4;               // units published ahead by the scheduling thread
+constexpr int kSchedConsumers = 15;         // warps that read each published unit (all but the scheduler's)
 
 enum : int { kErrTimeoutQ = 0x100, kErrTimeoutK = 0x200, kErrTimeoutS = 0x400, kErrTimeoutP = 0x800,
              kErrTimeoutPV = 0x1000, kErrTimeoutKEmpty = 0x2000, kErrTimeoutV = 0x4000,
-             kErrTimeoutVEmpty = 0x8000, kErrTimeoutQEmpty = 0x10000, kErrTimeoutMerge = 0x20000, kErrSmemAlign = 0x40000 };
+             kErrTimeoutVEmpty = 0x8000, kErrTimeoutQEmpty = 0x10000, kErrTimeoutMerge = 0x20000, kErrSmemAlign = 0x40000,
+             kErrTimeoutSched = 0x80000 };
 
 template <int D>
 struct TcSmem {
@@ -75,6 +79,8 @@ struct TcBars {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t drain;
+  uint64_t sched_full[kSchedRing], sched_empty[kSchedRing];
+  int sched_slot[kSchedRing];   // the CTA's n-th unit in slot n % kSchedRing
   uint32_t tmem_base;
   int abort_flag;
   int merge_old[2];   // per softmax warpgroup: arrivals seen by its unit's merge counter
@@ -141,9 +147,39 @@ DMA_DEVINL Unit unit_of(const FwdSchedule& sc, int u) {
   const int idx = u - sc.g[g].start, S = sc.g[g].S;
   return Unit{idx / S, sc.g[g].kp, idx % S, S, S > 1 ? sc.g[g].slot + idx : -1};
 }
-// The r-th unit of CTA c among G: snake order over the CTAs, so that the CTAs that took the heavier
-// units of one round take the lighter ones of the next.
-DMA_DEVINL int unit_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+// Dynamic schedule: the CTAs take the units (ordered heaviest first) from a global counter as they
+// finish earlier ones, the greedy longest-first assignment, which balances the SMs by the units'
+// actual durations.  In each CTA one thread (lane 0 of the first Q/K producer warp, the role that
+// runs ahead) takes the next unit and publishes it in a ring of kSchedRing slots; every other warp
+// reads unit n from slot n % kSchedRing and releases the slot.  The counter ends above n_units;
+// the last CTA to finish resets it (and the list kernel zeroes it with the mask).
+DMA_DEVINL int sched_publish(TcBars& bar, int n, int32_t* ctr, int n_units, volatile int* abort_flag,
+                             int32_t* status) {
+  const int slot = n % kSchedRing;
+  if (n >= kSchedRing &&
+      !tc::mbar_wait(&bar.sched_empty[slot], ((n / kSchedRing) - 1) & 1, abort_flag, status, kErrTimeoutSched))
+    return -1;
+  int u = atomicAdd(ctr, 1);
+  if (u > n_units) u = n_units;
+  bar.sched_slot[slot] = u;
+  tc::mbar_arrive(&bar.sched_full[slot]);
+  return u;
+}
+DMA_DEVINL int sched_take(TcBars& bar, int n, volatile int* abort_flag, int32_t* status) {
+  const int slot = n % kSchedRing;
+  if (!tc::mbar_wait(&bar.sched_full[slot], (n / kSchedRing) & 1, abort_flag, status, kErrTimeoutSched)) return -1;
+  const int u = *reinterpret_cast<volatile int*>(&bar.sched_slot[slot]);
+  tc::mbar_arrive(&bar.sched_empty[slot]);
+  return u;
+}
+// Warp-collective: lane 0 publishes (the scheduling warp) or takes unit n; every lane gets it.
+DMA_DEVINL int sched_unit_warp(TcBars& bar, int n, bool scheduler, int32_t* ctr, int n_units,
+                               volatile int* abort_flag, int32_t* status) {
+  int u = -1;
+  if ((threadIdx.x & 31) == 0)
+    u = scheduler ? sched_publish(bar, n, ctr, n_units, abort_flag, status) : sched_take(bar, n, abort_flag, status);
+  return __shfl_sync(0xffffffffu, u, 0);
+}
 // Tiles [tb, te) of the unit's pair list of n_live entries.
 DMA_DEVINL void unit_tiles(const Unit& x, int n_live, int& tb, int& te) {
   const int n = (n_live + kTcBK - 1) / kTcBK;
@@ -158,7 +194,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
                    const int32_t* __restrict__ pcounts, const int32_t* __restrict__ plists,
                    const int32_t* __restrict__ plen, const float* __restrict__ pdl, OutT* __restrict__ O,
                    float* __restrict__ LSE, float* __restrict__ fpart, float* __restrict__ fml,
-                   int32_t* __restrict__ fcnt, int32_t* __restrict__ status, int H, int G, int N, int n_pairs,
+                   int32_t* __restrict__ fcnt, int32_t* __restrict__ sched_ctr, int32_t* __restrict__ status, int H,
+                   int G, int N, int n_pairs,
                    int pair_cap, float scale_log2, int q0) {
   using S = TcSmem<D>;
   const int Nq = N - q0;   // the queries are positions [q0, N) (q0 > 0: a chunk of a longer sequence)
@@ -166,7 +203,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   TcBars& bar = *reinterpret_cast<TcBars*>(sm + S::kBars);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_units = sched.n_units;
-  const int cta = blockIdx.x, n_ctas = gridDim.x;
   volatile int* abort_flag = &bar.abort_flag;
 
   if (tid == 0) {
@@ -185,6 +221,10 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       tc::mbar_init(&bar.pv_done[i], 1);
     }
     tc::mbar_init(&bar.drain, 1);
+    for (int i = 0; i < kSchedRing; ++i) {
+      tc::mbar_init(&bar.sched_full[i], 1);
+      tc::mbar_init(&bar.sched_empty[i], kSchedConsumers);
+    }
     tc::fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -223,7 +263,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       int n_done = 0;              // items done (Q buffer phase)
       bool ok = !*abort_flag;
       for (int r = 0; ok; ++r) {
-        const int u = unit_index(r, cta, n_ctas);
+        const int u = sched_unit_warp(bar, r, warp == kKWarp0, sched_ctr, n_units, abort_flag, status);
+        if (u < 0) {
+          ok = false;
+          break;
+        }
         if (u >= n_units) break;
         const Unit it = unit_of(sched, u);
         const size_t lbase = ((size_t)it.bh * n_pairs + it.kp) * pair_cap;
@@ -292,7 +336,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         int n_done = 0;            // items done
         bool ok = !*abort_flag;
         for (int r = 0; ok; ++r) {
-          const int u = unit_index(r, cta, n_ctas);
+          const int u = sched_take(bar, r, abort_flag, status);
+          if (u < 0) {
+            ok = false;
+            break;
+          }
           if (u >= n_units) break;
           const Unit it = unit_of(sched, u);
           int tb, te;
@@ -364,7 +412,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
     int tcount = 0;
     bool ok = !*abort_flag;
     for (int rr = 0; ok; ++rr) {
-      const int u = unit_index(rr, cta, n_ctas);
+      const int u = sched_unit_warp(bar, rr, false, sched_ctr, n_units, abort_flag, status);
+      if (u < 0) {
+        ok = false;
+        break;
+      }
       if (u >= n_units) break;
       const Unit it = unit_of(sched, u);
       const int32_t* cnt = pcounts + ((size_t)it.bh * n_pairs + it.kp) * 2;
@@ -616,6 +668,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
   __syncthreads();
   tc::fence_after();
   if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
+  if (tid == 0) {   // the last CTA to finish leaves the schedule's counters at zero for the next launch
+    __threadfence();
+    if (atomicAdd(sched_ctr + 1, 1) == (int)gridDim.x - 1) {
+      sched_ctr[0] = 0;
+      sched_ctr[1] = 0;
+    }
+  }
 }
 
 template <int D, typename OutT>
@@ -639,6 +698,7 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
                                    ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
                                    ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE, ws_ptr<float>(ws, P.off_fpart),
                                    ws_ptr<float>(ws, P.off_fml), ws_ptr<int32_t>(ws, P.off_fcnt),
+                                   ws_ptr<int32_t>(ws, P.off_fcnt) + (size_t)P.B * P.H * P.n_pairs * 4,
                                    ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_pairs, P.pair_cap,
                                    P.scale * kLog2e, P.q0);
   return cudaGetLastError();

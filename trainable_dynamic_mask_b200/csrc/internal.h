@@ -65,7 +65,8 @@ struct Plan {
   // e_j - j (i32) and delta_j * log2(e) (f32); [B, H, n_pairs, pair_cap], counts [.., 2]
   size_t off_pcounts, off_plists, off_plen, off_pdl;
   // attention forward split units: partial O [slot][half][D][128] f32, (m, l) [slot][half][2][128]
-  // f32, and per pair [arrivals, partials written] x 2 halves (i32, zeroed by the list kernel)
+  // f32, and per pair [arrivals, partials written] x 2 halves (i32, zeroed by the list kernel),
+  // followed by the dynamic schedule's [next unit, CTAs done] (i32, zeroed likewise)
   size_t off_fpart, off_fml, off_fcnt;
   FwdSchedule sched;
   size_t off_gx;                       // gate backward: gx [B, H, N] f32

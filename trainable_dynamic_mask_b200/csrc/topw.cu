@@ -389,6 +389,8 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
   int nfull[3] = {0, 0, 0}, npart[3] = {0, 0, 0};
   // the attention forward's merge counters of this pair start at zero for every new mask
   if (tid < 4) fcnt[((size_t)row * n_pairs + kp) * 4 + tid] = 0;
+  // and its dynamic schedule's counters (after the merge counters of every pair)
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid < 2) fcnt[(size_t)gridDim.y * n_pairs * 4 + tid] = 0;
   // e_j and delta_j of this thread's 4 keys, loaded one round ahead
   int enext[4];
   float dnext[4];
