@@ -266,6 +266,16 @@ dma_status_t dma_check_device_status(const dma_params_t* p, void* workspace, voi
                                      int32_t* code);
 dma_status_t dma_clear_device_status(const dma_params_t* p, void* workspace, void* stream);
 
+/*
+ * Check of the device-side failure path: launches one thread that waits on a barrier nothing
+ * completes, with a limit of limit_cycles SM clocks (1 .. 2^34), after which it gives up, ORs
+ * status bit 0x1 into the workspace status word and returns.  dma_check_device_status then reports
+ * DMA_ERR_TIMEOUT; clear the word afterwards.  The same bounded wait guards every wait of the
+ * tcgen05 kernels (there with a limit of about two seconds).
+ */
+dma_status_t dma_selftest_bounded_wait(const dma_params_t* p, void* workspace, size_t workspace_bytes,
+                                       int64_t limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -146,6 +146,10 @@ assert lib.dma_attn_bwd(ctypes.byref(pc), *args) == UNSUPPORTED
 assert lib.dma_topk_append(pp, FAKE, FAKE, need, None) == INVALID
 assert lib.dma_topk_append(ctypes.byref(pd), None, FAKE, needd, None) == INVALID
 assert lib.dma_topk_append(ctypes.byref(pd), FAKE, FAKE, needd - 1, None) == WORKSPACE
+# selftest_bounded_wait(p, ws, ws_bytes, limit_cycles, stream): the limit is checked first
+assert lib.dma_selftest_bounded_wait(pp, FAKE, need, 0, None) == INVALID
+assert lib.dma_selftest_bounded_wait(pp, FAKE, need, 1 << 40, None) == INVALID
+assert lib.dma_selftest_bounded_wait(pp, FAKE, need - 1, 1000, None) == WORKSPACE
 # gate_append(p, V, Delta, A, delta, x_save, stream)
 assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, None, None, None) == INVALID
 assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE + 4, None) == INVALID

@@ -20,7 +20,8 @@ __all__ = [
     "BLOCK_Q", "DMA_BF16", "DMA_F32", "DmaError", "DmaParams", "LIB_PATH", "load", "exported_names",
     "make_params", "workspace_size", "workspace_layout", "gate", "topk_mask", "topk_append", "gate_append",
     "attn_fwd", "attn_bwd",
-    "gate_bwd", "gate_bwd_noalloc", "check_device_status", "clear_device_status", "abi_version", "alloc_workspace", "forward",
+    "gate_bwd", "gate_bwd_noalloc", "check_device_status", "clear_device_status", "selftest_bounded_wait",
+    "abi_version", "alloc_workspace", "forward",
     "backward",
 ]
 
@@ -128,6 +129,13 @@ def check_device_status(p, workspace, stream=None) -> int:
     code = ctypes.c_int32(0)
     load().dma_check_device_status(ctypes.byref(p), _ptr(workspace), _stream(stream), ctypes.byref(code))
     return int(code.value)
+
+
+def selftest_bounded_wait(p, workspace, limit_cycles=1_000_000, stream=None):
+    """Launch the device-side bounded-wait check (a wait that must give up and report)."""
+    check("dma_selftest_bounded_wait", load().dma_selftest_bounded_wait(ctypes.byref(p), _ptr(workspace),
+                                                                        _nbytes(workspace), int(limit_cycles),
+                                                                        _stream(stream)))
 
 
 def clear_device_status(p, workspace, stream=None):

@@ -56,6 +56,7 @@ _SIGS = {
                              c_vp],
     "dma_check_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp, ctypes.POINTER(c_i32)],
     "dma_clear_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp],
+    "dma_selftest_bounded_wait": [ctypes.POINTER(DmaParams), c_vp, c_sz, ctypes.c_int64, c_vp],
 }
 _RESTYPES = {"dma_status_string": ctypes.c_char_p, "dma_abi_version": c_i32}
 

@@ -398,6 +398,16 @@ dma_status_t dma_check_device_status(const dma_params_t* p, void* workspace, voi
   return v == 0 ? DMA_OK : DMA_ERR_TIMEOUT;
 }
 
+dma_status_t dma_selftest_bounded_wait(const dma_params_t* p, void* workspace, size_t workspace_bytes,
+                                       int64_t limit_cycles, void* stream) {
+  Plan P;
+  dma_status_t st = make_plan(p, &P);
+  if (st != DMA_OK) return st;
+  if (limit_cycles < 1 || limit_cycles > ((int64_t)1 << 34)) return DMA_ERR_INVALID_ARG;
+  if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
+  return cuda_status(launch_selftest_wait(P, workspace, (long long)limit_cycles, (cudaStream_t)stream));
+}
+
 dma_status_t dma_clear_device_status(const dma_params_t* p, void* workspace, void* stream) {
   Plan P;
   dma_status_t st = make_plan(p, &P);

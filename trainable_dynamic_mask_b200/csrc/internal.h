@@ -97,6 +97,7 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
                                 cudaStream_t s);
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s);
 cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s);
+cudaError_t launch_selftest_wait(const Plan& P, void* ws, long long limit_cycles, cudaStream_t s);
 cudaError_t launch_gate_append(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,
                                float* x_save, cudaStream_t s);
 cudaError_t launch_convert_f32_to_bf16(const float* src, uint16_t* dst, size_t n, cudaStream_t s);
