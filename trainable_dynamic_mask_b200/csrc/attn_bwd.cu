@@ -19,18 +19,52 @@ namespace dma {
 namespace {
 
 // ---------------------------------------------------------------- D = rowsum(dO * O)
+// One warp per kRowdotRows rows; each lane reads 4 consecutive elements of O and of dO per row (8- or
+// 16-byte loads), the loads of all the warp's rows issued before the sums.
+DMA_DEVINL void load4_f32(const uint16_t* p, float (&v)[4]) {
+  const uint2 w = *reinterpret_cast<const uint2*>(p);
+  v[0] = __uint_as_float(w.x << 16);
+  v[1] = __uint_as_float(w.x & 0xffff0000u);
+  v[2] = __uint_as_float(w.y << 16);
+  v[3] = __uint_as_float(w.y & 0xffff0000u);
+}
+DMA_DEVINL void load4_f32(const float* p, float (&v)[4]) {
+  const float4 w = *reinterpret_cast<const float4*>(p);
+  v[0] = w.x;
+  v[1] = w.y;
+  v[2] = w.z;
+  v[3] = w.w;
+}
+
+constexpr int kRowdotRows = 4;   // rows per warp, loaded together
+
 template <typename OT>
 __global__ void bwd_rowdot_kernel(const OT* __restrict__ O, const uint16_t* __restrict__ dO,
                                   float* __restrict__ Drow, size_t rows, int D) {
-  const size_t r = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const size_t r0 = ((size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * kRowdotRows;
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
-  float acc = 0.f;
-  for (int c = lane; c < D; c += 32)
-    acc = fmaf(load_as_f32(O + r * D + c), bf16_to_f32(dO[r * D + c]), acc);
+  if (r0 >= rows) return;
+  float acc[kRowdotRows];
+  for (int c = lane * 4; c < D; c += 128) {
+    float o[kRowdotRows][4], g[kRowdotRows][4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) Drow[r] = acc;
+    for (int k = 0; k < kRowdotRows; ++k) {
+      const size_t r = r0 + k < rows ? r0 + k : r0;
+      load4_f32(O + r * D + c, o[k]);
+      load4_f32(dO + r * D + c, g[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kRowdotRows; ++k)
+      acc[k] = fmaf(o[k][0], g[k][0], fmaf(o[k][1], g[k][1], fmaf(o[k][2], g[k][2],
+                    fmaf(o[k][3], g[k][3], c == lane * 4 ? 0.f : acc[k]))));
+  }
+#pragma unroll
+  for (int k = 0; k < kRowdotRows; ++k) {
+    float v = lane * 4 < D ? acc[k] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0 && r0 + k < rows) Drow[r0 + k] = v;
+  }
 }
 
 template <int D, typename OutT>
@@ -40,7 +74,9 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
                          float* d_delta, cudaStream_t s) {
   float* Drow = ws_ptr<float>(ws, P.off_rowD);
   const size_t rows = (size_t)P.B * P.H * P.N;
-  bwd_rowdot_kernel<OutT><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>((const OutT*)O, dO, Drow, rows, D);
+  const size_t per_block = 8 * kRowdotRows;
+  bwd_rowdot_kernel<OutT><<<(unsigned)((rows + per_block - 1) / per_block), 256, 0, s>>>((const OutT*)O, dO, Drow,
+                                                                                       rows, D);
   {
     cudaError_t e = launch_bwd_dq_tc(P, Q, K, V, dO, delta, evict, ws, LSE, Drow, dQ, s);
     if (e != cudaSuccess) return e;
