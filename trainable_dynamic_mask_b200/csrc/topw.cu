@@ -535,7 +535,7 @@ topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ d
 
 // ---------------------------------------------------------------- decode selection
 
-constexpr int kSelThreads = 1024;
+constexpr int kSelThreads = 512;                // two CTAs per SM: a row per CTA, all rows in one wave
 constexpr int kSelBatch = 8;                   // rounds of loads issued together
 constexpr int kSelBits = 12;                   // histogram window
 constexpr int kSelBins = 1 << kSelBits;
@@ -593,7 +593,7 @@ DMA_DEVINL void sel_find_bin(SelShared& S, uint32_t need, int nbins, int tid) {
 // would separate almost nothing).  Passes over the row narrow the window until the bin holding the
 // w-th best key has at most kSelCand keys; those are then resolved in shared memory.  A last pass
 // writes the selected positions in ascending order.
-__global__ void __launch_bounds__(kSelThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, 2)
 topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int N, int w) {
   extern __shared__ __align__(16) unsigned char sel_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(sel_raw);
