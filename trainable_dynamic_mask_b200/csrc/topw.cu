@@ -159,35 +159,48 @@ topw_thresh_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__
     }
   }
   __syncthreads();
-  for (int k = warp; k <= nch; k += kThWarps) {
+  // boundaries with kC <= w evict nothing (T = N); warps take the others, from the first
+  for (int k = tid; k <= nch; k += kThThreads)
+    if (min(k * kC, N) <= w) T_out[(size_t)row * cw + k] = N;
+  const int kfirst = N > w ? w / kC + 1 : nch + 1;   // first k with kC > w
+  for (int k = kfirst + warp; k <= nch; k += kThWarps) {
     const int Pk = min(k * kC, N);
-    int Tk = N;
-    if (Pk > w) {
-      int before = 0, rbs = -1;
-      for (int rb0 = 0; rb0 < nch && rbs < 0; rb0 += 32) {
-        const int rb = rb0 + lane;
-        const int v = rb < nch ? (int)table[rb * cw + k] : 0;
-        int incl = v;
+    int before = 0, rbs = -1;
+    for (int rb0 = 0; rb0 < nch && rbs < 0; rb0 += 32) {
+      const int rb = rb0 + lane;
+      const int v = rb < nch ? (int)table[rb * cw + k] : 0;
+      int incl = v;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const uint32_t hit = __ballot_sync(0xffffffffu, before + incl >= w);
-        if (hit) {
-          const int l = __ffs(hit) - 1;
-          rbs = rb0 + l;
-          before += __shfl_sync(0xffffffffu, incl - v, l);
-        } else {
-          before += __shfl_sync(0xffffffffu, incl, 31);
-        }
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
       }
-      int need = w - before;
-      for (int r0 = rbs * 128; r0 < min(rbs * 128 + 128, N); r0 += 32) {
-        const int r = r0 + lane;
-        const uint32_t m = __ballot_sync(0xffffffffu, r < N && prow[min(r, N - 1)] < Pk);
-        const int c = __popc(m);
-        if (c >= need) { Tk = r0 + nth_set_bit(m, need - 1); break; }
+      const uint32_t hit = __ballot_sync(0xffffffffu, before + incl >= w);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        rbs = rb0 + l;
+        before += __shfl_sync(0xffffffffu, incl - v, l);
+      } else {
+        before += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    // the w-th key with position < Pk lies in rank bucket rbs: its 128 positions, loaded together
+    const int rend = min(rbs * 128 + 128, N);
+    int pos[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = rbs * 128 + 32 * u + lane;
+      pos[u] = r < rend ? prow[r] : INT_MAX;
+    }
+    int need = w - before, Tk = N;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t m = __ballot_sync(0xffffffffu, pos[u] < Pk);
+      const int c = __popc(m);
+      if (need > 0 && c >= need) {
+        Tk = rbs * 128 + 32 * u + nth_set_bit(m, need - 1);
+        need = 0;
+      } else if (need > 0) {
         need -= c;
       }
     }
@@ -209,7 +222,7 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
                   const int32_t* __restrict__ T_in, int32_t* __restrict__ evict, int32_t* __restrict__ status,
                   int N, int w) {
   constexpr int kEvU = 4;            // ranks scanned per thread per round
-  __shared__ int32_t crank[kC];      // ranks of the chunk's own keys
+  __shared__ __align__(16) int32_t crank[kC];   // ranks of the chunk's own keys (INT_MAX past the end)
   __shared__ int32_t L[kC];          // old candidates, ascending rank
   __shared__ int32_t Lpos[kC];       // their positions
   __shared__ int32_t wcount[kEvU][kEvThreads / 32];
@@ -223,7 +236,7 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   int32_t* erow = evict + (size_t)row * N;
   const int Ta = T[k], Tb = T[k + 1], Tf = T[nch];
   const int Sk = min(t0, w);
-  if (tid < t1 - t0) crank[tid] = rrow[t0 + tid];
+  crank[tid] = tid < t1 - t0 ? rrow[t0 + tid] : INT_MAX;
   // old candidates in rank order: the ranks in (Tb, Ta] held by positions < t0; all loads of a round
   // are issued before its ballots
   int nL = 0;
@@ -269,21 +282,55 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   }
   __syncthreads();
   // The chunk's keys in rank order, and pmask[q] = offsets (t - t0) of the chunk's q best keys:
-  // the chunk keys better than rank r are pmask[#{chunk ranks < r}].
+  // the chunk keys better than rank r are pmask[#{chunk ranks < r}].  pmask is the exclusive
+  // prefix OR, over the chunk ranks q, of the one-bit mask of the offset holding rank q.
   __shared__ int32_t srank[kC];
+  __shared__ int32_t soff[kC];
   __shared__ uint32_t pmask[kC + 1][kEvThreads / 32];
+  __shared__ uint32_t wor[kEvThreads / 32][kEvThreads / 32];
+  static_assert(kEvThreads == kC, "one thread per chunk offset");
   const int nc = t1 - t0;
   int cr = kC;   // rank of offset tid among the chunk's keys
   if (tid < nc) {
     const int my = crank[tid];
     int q = 0;
-    for (int i = 0; i < nc; ++i) q += crank[i] < my;
+    const int4* c4 = reinterpret_cast<const int4*>(crank);
+#pragma unroll 8
+    for (int i = 0; i < kC / 4; ++i) {
+      const int4 v = c4[i];
+      q += (v.x < my) + (v.y < my) + (v.z < my) + (v.w < my);
+    }
     cr = q;
     srank[q] = my;
+    soff[q] = tid;
   }
-  for (int q = 0; q <= nc; ++q) {
-    const uint32_t m = __ballot_sync(0xffffffffu, cr < q);   // word `warp`: offsets 32 warp + lane
-    if (lane == 0) pmask[q][warp] = m;
+  __syncthreads();
+  {
+    // thread q: one-bit mask of the offset of chunk rank q, then an inclusive OR scan over q
+    uint32_t v[kEvThreads / 32];
+    const int o = tid < nc ? soff[tid] : -1;
+#pragma unroll
+    for (int wd = 0; wd < kEvThreads / 32; ++wd) v[wd] = (o >> 5) == wd ? 1u << (o & 31) : 0u;
+#pragma unroll
+    for (int sh = 1; sh < 32; sh <<= 1) {
+#pragma unroll
+      for (int wd = 0; wd < kEvThreads / 32; ++wd) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v[wd], sh);
+        if (lane >= sh) v[wd] |= y;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int wd = 0; wd < kEvThreads / 32; ++wd) wor[warp][wd] = v[wd];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int wd = 0; wd < kEvThreads / 32; ++wd) {
+      uint32_t acc = v[wd];
+      for (int i = 0; i < warp; ++i) acc |= wor[i][wd];
+      pmask[tid + 1][wd] = acc;
+      if (tid == 0) pmask[0][wd] = 0u;
+    }
   }
   __syncthreads();
   const int ncand = nL + (t1 - t0);
