@@ -341,44 +341,22 @@ gate_fwd_mma_kernel(const uint16_t* __restrict__ V, const uint16_t* __restrict__
   const int b = blockIdx.y, p0 = blockIdx.x * kGmP;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dch = d / 8;
-  // ---- stage V (16 positions x K) and Delta (K x H, padded to 8 HT columns)
-  // batches of kGmBatch 16-byte loads per thread, all issued before their stores
-  constexpr int kGmBatch = 8;
-  for (int q0 = 0; q0 < kGmP * KC; q0 += kGmBatch * kGmThreads) {
-    uint4 v[kGmBatch];
-#pragma unroll
-    for (int u = 0; u < kGmBatch; ++u) {
-      const int q = q0 + u * kGmThreads + tid;
-      const int p = q / KC, kc = q % KC;
-      const int g = kc / dch, c = kc % dch;
-      const int pos = p0 + p;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (q < kGmP * KC && pos < N) v[u] = *reinterpret_cast<const uint4*>(V + ((size_t)(b * Hkv + g) * N + pos) * d + c * 8);
-    }
-#pragma unroll
-    for (int u = 0; u < kGmBatch; ++u) {
-      const int q = q0 + u * kGmThreads + tid;
-      const int p = q / KC, kc = q % KC;
-      if (q < kGmP * KC) *reinterpret_cast<uint4*>(Vs + (size_t)p * K + ((kc ^ (p & 7)) * 8)) = v[u];
-    }
+  // ---- stage V (16 positions x K) and Delta (K x H, padded to 8 HT columns): every 16-byte
+  // copy of both is issued before the first wait (one memory round trip)
+  for (int q = tid; q < kGmP * KC; q += kGmThreads) {
+    const int p = q / KC, kc = q % KC;
+    const int g = kc / dch, c = kc % dch;
+    const int pos = p0 + p;
+    const bool in = pos < N;
+    const uint16_t* src = in ? V + ((size_t)(b * Hkv + g) * N + pos) * d + c * 8 : V;
+    cp_async_16(smem_u32(Vs + (size_t)p * K + ((kc ^ (p & 7)) * 8)), src, in ? 16 : 0);
   }
   if ((H & 7) == 0) {
     const int hc = H / 8;
-    for (int q0 = 0; q0 < K * HT; q0 += kGmBatch * kGmThreads) {
-      uint4 v[kGmBatch];
-#pragma unroll
-      for (int u = 0; u < kGmBatch; ++u) {
-        const int q = q0 + u * kGmThreads + tid;
-        const int r = q / HT, c = q % HT;
-        v[u] = make_uint4(0, 0, 0, 0);
-        if (q < K * HT && c < hc) v[u] = *reinterpret_cast<const uint4*>(Delta + (size_t)r * H + c * 8);
-      }
-#pragma unroll
-      for (int u = 0; u < kGmBatch; ++u) {
-        const int q = q0 + u * kGmThreads + tid;
-        const int r = q / HT, c = q % HT;
-        if (q < K * HT) *reinterpret_cast<uint4*>(Ds + (size_t)r * 8 * HT + c * 8) = v[u];
-      }
+    for (int q = tid; q < K * HT; q += kGmThreads) {
+      const int r = q / HT, c = q % HT;
+      const bool in = c < hc;
+      cp_async_16(smem_u32(Ds + (size_t)r * 8 * HT + c * 8), in ? Delta + (size_t)r * H + c * 8 : Delta, in ? 16 : 0);
     }
   } else {
     for (int q = tid; q < K * 8 * HT; q += kGmThreads) {
@@ -386,6 +364,8 @@ gate_fwd_mma_kernel(const uint16_t* __restrict__ V, const uint16_t* __restrict__
       Ds[q] = h < H ? Delta[(size_t)r * H + h] : (uint16_t)0;
     }
   }
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
   // ---- partial products over this warp's reduction steps
   float acc[HT][4];
