@@ -15,10 +15,13 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every call is asynchronous on the caller's CUDA stream (`stream` is a cudaStream_t passed
- *    as void*; NULL is the legacy default stream).  No call synchronises the host, allocates
- *    device memory, or keeps a pointer after its stream work completes.  The library has no
- *    mutable global state; calls on different streams may run concurrently when their buffers
- *    (including workspaces) are distinct.
+ *    as void*; NULL is the legacy default stream).  No call allocates device memory or keeps a
+ *    pointer after its stream work completes, and none synchronises the host except
+ *    dma_check_device_status, which reads the workspace status word back.  The library's only
+ *    global state is a host-side record, per kernel and device, that the kernel's shared-memory
+ *    limit has been raised (kept behind a mutex), and the fixed scratch array of
+ *    dma_gate_bwd_noalloc.  Calls on different streams may run concurrently when their buffers
+ *    (including workspaces) are distinct; dma_gate_bwd_noalloc calls must not overlap.
  *  - All pointers are device pointers, 16-byte aligned, to dense row-major (C-contiguous)
  *    tensors with the layouts given per argument.  The caller owns every buffer.
  *  - Arguments are validated before anything is launched.  On any error nothing is launched
@@ -160,8 +163,8 @@ dma_status_t dma_gate(const dma_params_t* p, const void* V, const void* Delta, c
  *          iff j <= t < e_j; e_j == j means key j is never selected.  Because delta does not
  *          depend on the query, the queries selecting a key always form this interval.
  *          Also writes the per-block live-key lists and counts into the workspace, and beside
-          each list entry the values the attention forward needs for that key (e_j and delta_j),
-          so that its load stage reads them with contiguous loads instead of a gather.
+ *          each list entry the values the attention forward needs for that key (e_j and delta_j),
+ *          so that its load stage reads them with contiguous loads instead of a gather.
  *          Decode (Nq == 1): `evict` must be NULL; the selected keys of the query at
  *          position N-1 are written to the workspace region off_sel.
  */
