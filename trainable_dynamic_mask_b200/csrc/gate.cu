@@ -324,8 +324,9 @@ __global__ void gate_bwd_reduce_kernel(const float* __restrict__ part, const flo
 // positions of one batch row, 8 warps splitting the reduction in 16-wide steps (step s to warp
 // s % 8); the 8 partial [16 x H] tiles are summed through shared memory.  The V rows of the 16
 // positions (all Hkv heads: 16 rows of Hkv*d) and Delta (zero-padded to HT*8 columns) are staged
-// with coalesced 16-byte loads; A fragments come from a 16-byte-chunk XOR swizzle (conflict-free
-// ldmatrix), B fragments from ldmatrix.trans of the row-major Delta.
+// with coalesced 16-byte async copies, all issued before one wait; A fragments come from a
+// 16-byte-chunk XOR swizzle (conflict-free ldmatrix), B fragments from ldmatrix.trans of the
+// row-major Delta.
 constexpr int kGmP = 16;
 constexpr int kGmThreads = 256;
 
