@@ -92,7 +92,8 @@ typedef enum {
  *   dtype  a dma_dtype_t
  *
  * Limits of this implementation (DMA_ERR_UNSUPPORTED beyond them): prefill/training
- * N <= 16384; decode N <= 1<<24 and min(w, N) <= 4096 * d; B*H <= 65535; d in {64, 128}.
+ * N <= 16384; decode N <= 1<<24 and min(w, N) <= 4096 * d; B*H <= 65535; d in {64, 128};
+ * dma_gate, dma_gate_bwd and dma_gate_bwd_noalloc: H <= 64.
  */
 typedef struct {
   int32_t B, H, Hkv, N, Nq, d, w;
@@ -245,14 +246,17 @@ dma_status_t dma_gate_bwd(const dma_params_t* p, const void* V, const void* Delt
  * counterpart of this entry point; it exists for those callers only.
  *
  * Arguments and results are those of dma_gate_bwd (outputs within the same tolerance), except
- * that there is no workspace: the scratch (gx and the partial sums of dA and dDelta, about
- * 4 * (B*H*N + ceil(N/512)*B*Hkv*d*H) bytes) lives in a fixed array of DMA_NOALLOC_SCRATCH_BYTES
- * that the library reserves on every GPU that loads it, until the process exits.  A problem whose
- * scratch does not fit returns DMA_ERR_UNSUPPORTED before anything is launched.  The first call
- * on a device looks the array's device address up (cudaGetSymbolAddress) with that device
- * current, so make that first call before any stream capture.  All calls share the one array:
- * calls whose GPU work overlaps (on different streams or from different host threads on one
- * device) race on it, so the caller must serialise them.  Nothing is allocated or freed.
+ * that there is no workspace: the scratch (gx, the partial sums of dA and those of dDelta) lives in
+ * a fixed array of DMA_NOALLOC_SCRATCH_BYTES that the library reserves on every GPU that loads it,
+ * until the process exits.  With a(x) = x rounded up to a multiple of 256, a problem needs
+ *     a(4*B*H*N) + a(4*B*H*ceil(N/1024)) + a(4*ceil(N/512)*B*Hkv*d*H)
+ * bytes of it; one that needs more returns DMA_ERR_UNSUPPORTED before anything is launched.
+ * The first call on a device (and the first after a device reset, which gives the device a new
+ * context) looks the array's device address up (cudaGetSymbolAddress) with that device current,
+ * so make that first call before any stream capture.  All calls share the one array: calls whose
+ * GPU work overlaps (on different streams or from different host threads on one device) race on
+ * it, so the caller must serialise them.  Every scratch element a call reads is written by that
+ * call first.  Nothing is allocated or freed.
  */
 #define DMA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 dma_status_t dma_gate_bwd_noalloc(const dma_params_t* p, const void* V, const void* Delta,

@@ -155,6 +155,34 @@ assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, None, None, None)
 assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE + 4, None) == INVALID
 pdec = dma.make_params(8, 32, 8, 65536, 128, 2048, Nq=1)   # 64 MiB of gx alone: more than the fixed array
 assert lib.dma_gate_bwd_noalloc(ctypes.byref(pdec), *([FAKE] * 9), None) == UNSUPPORTED
+# the gate kernels hold at most 64 query heads; more is refused on the host, not at launch
+ph = dma.make_params(1, 72, 8, 256, 128, 64)
+needh = need_of(ph)
+assert lib.dma_gate(ctypes.byref(ph), FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == UNSUPPORTED
+assert lib.dma_gate_bwd(ctypes.byref(ph), *([FAKE] * 9), FAKE, needh, None) == UNSUPPORTED
+assert lib.dma_gate_bwd_noalloc(ctypes.byref(ph), *([FAKE] * 9), None) == UNSUPPORTED
+# the scratch formula of dma_gate_bwd_noalloc, exact at the boundary of the fixed array: a problem that
+# fits passes every host check and only fails for want of a device (DMA_ERR_CUDA), one more position
+# does not fit (DMA_ERR_UNSUPPORTED)
+CUDA_ERR = 4
+a256 = lambda x: (x + 255) // 256 * 256
+cdiv = lambda x, y: (x + y - 1) // y
+def scratch(B, H, Hkv, N, d):
+    return a256(4 * B * H * N) + a256(4 * B * H * cdiv(N, 1024)) + a256(4 * cdiv(N, 512) * B * Hkv * d * H)
+LIMIT = 16 << 20
+found = 0
+for (B, H, Hkv, d) in ((1, 64, 8, 64), (3, 40, 8, 64), (2, 64, 4, 128)):
+    lo, hi = 1, 1 << 24   # largest N whose scratch fits
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if scratch(B, H, Hkv, mid, d) <= LIMIT: lo = mid
+        else: hi = mid - 1
+    for N, want in ((lo, CUDA_ERR), (lo + 1, UNSUPPORTED)):
+        q = dma.make_params(B, H, Hkv, N, d, 64, Nq=1)
+        got = lib.dma_gate_bwd_noalloc(ctypes.byref(q), *([FAKE] * 9), None)
+        assert got == want, (B, H, Hkv, d, N, got, want)
+    found += 1
+assert found == 3
 print("ok")
 """
 

@@ -271,6 +271,7 @@ dma_status_t dma_gate(const dma_params_t* p, const void* V, const void* Delta, c
   if (st != DMA_OK) return st;
   if (!ok_ptr(V) || !ok_ptr(Delta) || !ok_ptr(A) || !ok_ptr(delta)) return DMA_ERR_INVALID_ARG;
   if (x_save != nullptr && !aligned16(x_save)) return DMA_ERR_INVALID_ARG;
+  if (P.H > kGateMaxH) return DMA_ERR_UNSUPPORTED;
   return cuda_status(launch_gate_fwd(P, V, Delta, A, delta, x_save, (cudaStream_t)stream));
 }
 
@@ -377,6 +378,7 @@ dma_status_t dma_gate_bwd(const dma_params_t* p, const void* V, const void* Delt
   if (!ok_ptr(V) || !ok_ptr(Delta) || !ok_ptr(A) || !ok_ptr(x_save) || !ok_ptr(delta) ||
       !ok_ptr(d_delta) || !ok_ptr(dDelta) || !ok_ptr(dA) || !ok_ptr(dV_gate))
     return DMA_ERR_INVALID_ARG;
+  if (P.H > kGateMaxH) return DMA_ERR_UNSUPPORTED;
   if ((st = check_ws(P, workspace, workspace_bytes)) != DMA_OK) return st;
   return cuda_status(launch_gate_bwd(P, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate,
                                      workspace, (cudaStream_t)stream));

@@ -14,6 +14,7 @@ constexpr int kPairQ = 2 * kBlockQ;    // query rows per attention-forward work 
 constexpr int kTopwMaxN = 16384;      // prefill/training selection keeps a whole row in SMEM
 constexpr int kDecodeSplit = 256;      // selected keys per decode split (one per thread)
 constexpr int kGateSlice = 512;        // positions per partial sum of dDelta
+constexpr int kGateMaxH = 64;          // query heads the gate kernels hold in one register tile
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
