@@ -103,6 +103,10 @@ class ClockSampler:
             self.error = repr(e)
         self._t = threading.Thread(target=self._run, daemon=True)
 
+    def mark(self):
+        """Start of the timed region: samples from here on are also counted on their own."""
+        self._mark = len(self.samples)
+
     def _run(self):
         nv = self._nv
         while not self._stop.is_set():
@@ -132,8 +136,13 @@ class ClockSampler:
         if self._h is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "nvml")}
         reasons = sorted(self.reasons - {"gpu_idle"})
+        timed = self.samples[getattr(self, "_mark", 0):]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": reasons, "samples": len(self.samples)}
+                "reasons": reasons, "samples": len(self.samples),
+                "samples_in_timed_region": len(timed),
+                "sm_mhz_timed_region": statistics.median(timed) if timed else None,
+                "window": "the same step replayed untimed for --clock-soak seconds immediately before the "
+                          "timed region, then the timed region"}
 
 
 # ---------------------------------------------------------------- helpers
@@ -182,7 +191,8 @@ def run_ours(args, world, rank):
     peaks = _peaks()
     wl = get("prefill")
     I = make_inputs(wl)
-    p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype="bf16")
+    # an inference prefill: no backward follows, so the forward keeps nothing for one
+    p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype="bf16", forward_only=True)
     Q, K, V = (_to_dev_bf16(I.bits[n], torch) for n in ("Q", "K", "V"))
     Dl = _to_dev_bf16(I.bits["Delta"], torch)
     A = torch.from_numpy(I.A).cuda()
@@ -231,9 +241,24 @@ def run_ours(args, world, rank):
         attn = [e1.elapsed_time(e2) for e0, e1, e2 in evs]
         return step, attn
 
+    def soak(seconds):
+        # the same step, untimed, in batches until `seconds` have passed: the clock sampler needs a
+        # window longer than its sampling period, which a short timed region alone does not give
+        t0 = time.perf_counter()
+        with torch.cuda.stream(stream):
+            while time.perf_counter() - t0 < seconds:
+                for _ in range(200):
+                    flush.zero_()
+                    ga.replay()
+                    gb.replay()
+                stream.synchronize()
+
     timed(args.warmup)
     _barrier(world, torch)
     with ClockSampler(torch.cuda.current_device()) as clk:
+        soak(args.clock_soak)
+        _barrier(world, torch)
+        clk.mark()
         step_ms, attn_ms = timed(args.steps)
     _barrier(world, torch)
     total_ms = _max_over_ranks(sum(step_ms), world, torch)
@@ -242,10 +267,12 @@ def run_ours(args, world, rank):
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
     traffic = _traffic("attn_fwd_prefill", "attn_fwd_tc.cu")
+    torch.cuda.synchronize()
+    density = _pair_density(evict.cpu().numpy(), wl, np)
 
     # the same kernels with w = N (dense causal attention), timed the same way
     wl_d = wl.with_(w=wl.N)
-    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, dtype="bf16")
+    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, dtype="bf16", forward_only=True)
     ws_d = dma.alloc_workspace(p_d)
     O_d, LSE_d = torch.empty_like(O), torch.empty_like(LSE)
     with torch.cuda.stream(stream):
@@ -322,15 +349,18 @@ def run_ours(args, world, rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V, Delta ~ N(0, 0.02^2), A ~ U(-1, 0))",
-        "config": {"workload": "prefill", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N, "d": wl.d, "w": wl.w,
+        "config": {"workload": "prefill", "quoted_on": "the prefill configuration (the metric's own); the long "
+                   "prefill configuration is reported in legs.long",
+                   "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N, "d": wl.d, "w": wl.w,
                    "kept_pairs": wl.kept_pairs(), "step": "gate + top-w mask + attention forward",
+                   "forward_only": True,
                    "parallelism": f"replicas{world}", "l2": "flushed (256 MiB zeroed) before every step"},
         "roofline": {"kernel": "attn_fwd", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4), "peak_kind": "burst " + peaks["source"],
                      "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
                      "traffic": traffic, "avg_launch_us": round(attn_avg * 1e3, 2),
-                     "per_launch_flops": flops},
+                     "per_launch_flops": flops, "tile_density": density},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "api": "trainable_dynamic_mask_b200.forward"},
@@ -341,7 +371,7 @@ def run_ours(args, world, rank):
     }
     legs = [] if args.no_legs else [x for x in args.legs.split(",") if x]
     if legs:
-        run = {"decode": leg_decode, "train": leg_train, "chunk": leg_chunk}
+        run = {"decode": leg_decode, "train": leg_train, "chunk": leg_chunk, "long": leg_long}
         line["legs"] = {name: run[name](args, world, torch, dma, peaks) for name in legs}
         line["gpu_launches"] += sum(leg["gpu_launches"] for leg in line["legs"].values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -498,6 +528,118 @@ def leg_chunk(args, world, torch, dma, peaks):
             "gpu_launches": 7 * n}   # gate, top-w 5, attention
 
 
+def _pair_density(evict, wl, np):
+    """Executed-tile density of the attention forward: kept-pair FLOPs over the FLOPs of the
+    tensor-core tiles the kernel runs (each pair of 128-row blocks walks its live keys in tiles of
+    128; a key is live for the pair [t0, t1) when j < t1 and e_j > max(j, t0)).  Computed on the
+    host from the eviction indices the GPU wrote."""
+    e = evict.reshape(-1, wl.N)
+    j = np.arange(wl.N)
+    tiles = 0
+    for t0 in range(wl.q_pos0 // 256 * 256, wl.N, 256):
+        t1 = min(t0 + 256, wl.N)
+        live = ((j[None, :t1] < t1) & (e[:, :t1] > np.maximum(j[None, :t1], t0))).sum(axis=1)
+        tiles += int(((live + 127) // 128).sum())
+    executed = tiles * 128 * 256   # query rows x keys per tile
+    return {"kept_pairs": wl.kept_pairs(), "executed_pairs": executed,
+            "density": round(wl.kept_pairs() / executed, 4)}
+
+
+def leg_long(args, world, torch, dma, peaks):
+    """The long prefill workload (B=1, H=32, Hkv=8, N=16384, d=128, w=2048, 5% of key positions
+    scaled by 4): gate -> top-w mask -> attention forward, replayed from two CUDA graphs with L2
+    flushed before every step, the attention timed on its own for the roofline."""
+    import numpy as np
+
+    from workloads import get, make_inputs
+    wl = get("long")
+    I = make_inputs(wl)
+    p = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype="bf16", forward_only=True)
+    Q, K, V = (_to_dev_bf16(I.bits[n], torch) for n in ("Q", "K", "V"))
+    Dl = _to_dev_bf16(I.bits["Delta"], torch)
+    A = torch.from_numpy(I.A).cuda()
+    ws = dma.alloc_workspace(p)
+    delta = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device="cuda")
+    evict = torch.empty((wl.B, wl.H, wl.N), dtype=torch.int32, device="cuda")
+    O = torch.empty((wl.B, wl.H, wl.N, wl.d), dtype=torch.bfloat16, device="cuda")
+    LSE = torch.empty((wl.B, wl.H, wl.N), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flops = 4.0 * wl.d * wl.kept_pairs()
+    stream = torch.cuda.Stream()
+    s_ptr = stream.cuda_stream
+
+    def graphs(pp, w_ws, o, lse):
+        with torch.cuda.stream(stream):
+            dma.gate(pp, V, Dl, A, delta, None, w_ws, s_ptr)
+            dma.topk_mask(pp, delta, evict, w_ws, s_ptr)
+            dma.attn_fwd(pp, Q, K, V, delta, evict, w_ws, o, lse, s_ptr)
+            stream.synchronize()
+            ga, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(ga, stream=stream):
+                dma.gate(pp, V, Dl, A, delta, None, w_ws, s_ptr)
+                dma.topk_mask(pp, delta, evict, w_ws, s_ptr)
+            with torch.cuda.graph(gb, stream=stream):
+                dma.attn_fwd(pp, Q, K, V, delta, evict, w_ws, o, lse, s_ptr)
+        return ga, gb
+
+    def timed(ga, gb, n):
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for e0, e1, e2 in evs:
+                flush.zero_()
+                e0.record(stream)
+                ga.replay()
+                e1.record(stream)
+                gb.replay()
+                e2.record(stream)
+        stream.synchronize()
+        return sum(e0.elapsed_time(e2) for e0, e1, e2 in evs) / n, sum(e1.elapsed_time(e2) for e0, e1, e2 in evs) / n
+
+    ga, gb = graphs(p, ws, O, LSE)
+    n = max(5, min(args.steps, 100))
+    timed(ga, gb, args.warmup)
+    step_ms, attn_ms = timed(ga, gb, n)
+    step_ms = _max_over_ranks(step_ms, world, torch)
+    attn_ms = _max_over_ranks(attn_ms, world, torch)
+    torch.cuda.synchronize()
+    dens = _pair_density(evict.cpu().numpy(), wl, np)
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    del ga, gb
+    # the same kernels with w = N (dense causal), timed the same way
+    p_d = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.N, dtype="bf16", forward_only=True)
+    ws_d = dma.alloc_workspace(p_d)
+    gda, gdb = graphs(p_d, ws_d, O, LSE)
+    timed(gda, gdb, 2)
+    n_d = 5
+    step_d, attn_d = timed(gda, gdb, n_d)
+    step_d = _max_over_ranks(step_d, world, torch)
+    attn_d = _max_over_ranks(attn_d, world, torch)
+    del gda, gdb, ws_d
+    pairs_d = wl.with_(w=wl.N).kept_pairs()
+    flops_d = 4.0 * wl.d * pairs_d
+    dense = {"w": wl.N, "kept_pairs": pairs_d, "step_us": round(step_d * 1e3, 2), "attn_us": round(attn_d * 1e3, 2),
+             "attn_tflops": round(flops_d / (attn_d * 1e-3) / 1e12, 2),
+             "speedup_attn": round(attn_d / attn_ms, 3), "speedup_step": round(step_d / step_ms, 3), "steps": n_d}
+    out = {"metric": "long prefill kept-pair TFLOP/s (gate + top-w mask + attention forward)",
+           "value": round(world * flops / (step_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "config": {"workload": "long", "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N, "d": wl.d, "w": wl.w,
+                      "kept_pairs": wl.kept_pairs(), "scaled_key_positions": "5% x4", "forward_only": True,
+                      "l2": "flushed (256 MiB zeroed) before every step"},
+           "step_us": round(step_ms * 1e3, 2), "attn_us": round(attn_ms * 1e3, 2),
+           "roofline": {"kernel": "attn_fwd", "bound": "tensor", "achieved": round(achieved, 2),
+                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                        "peak_kind": "burst " + peaks["source"],
+                        "frac_of_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                        "traffic": _traffic("attn_fwd_long", "attn_fwd_tc.cu"), "avg_launch_us": round(attn_ms * 1e3, 2),
+                        "per_launch_flops": flops},
+           "tile_density": dens,
+           "dense_causal": dense,
+           "gpu_launches": 7 * n}
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds / 2, workload="long")
+    return out
+
+
 def leg_train(args, world, torch, dma, peaks):
     """Training step on the train workload: gate (saving x) + mask + attention
     forward + attention backward + gate backward.  kept-pair FLOPs = 14 d pairs
@@ -591,7 +733,7 @@ def _cpu_cores():
 
 def _oracle_sample(n_rows, wl, I, d32, e_cache, oracle, np):
     """Oracle forward on the first n_rows query rows (over heads, in order) of
-    the prefill workload; returns (seconds, kept-pair flops)."""
+    a prefill-type workload; returns (seconds, kept-pair flops)."""
     t0 = time.perf_counter()
     rows_left, flops = n_rows, 0.0
     for h in range(wl.H):
@@ -608,17 +750,17 @@ def _oracle_sample(n_rows, wl, I, d32, e_cache, oracle, np):
     return time.perf_counter() - t0, flops
 
 
-def cpu_baseline(budget_s=20.0):
-    """The oracle, as it stands, on the host cores: gate on the whole prefill
-    workload plus masked attention forward on as many query rows as fit the
-    time budget; kept-pair TFLOP/s of the rows processed."""
+def cpu_baseline(budget_s=20.0, workload="prefill"):
+    """The oracle, as it stands, on the host cores: gate on the whole workload
+    plus masked attention forward on as many query rows as fit the time
+    budget; kept-pair TFLOP/s of the rows processed."""
     import numpy as np
     from threadpoolctl import threadpool_limits
 
     import oracle
     from workloads import get, make_inputs
     cores = _cpu_cores()
-    wl = get("prefill")
+    wl = get(workload)
     I = make_inputs(wl)
     with threadpool_limits(limits=cores):
         t0 = time.perf_counter()
@@ -633,7 +775,7 @@ def cpu_baseline(budget_s=20.0):
     share = flops / (4.0 * wl.d * wl.kept_pairs())
     secs = t_rows + t_gate * share
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"prefill workload: float64 gate on all of V (cost charged pro rata) + top-w and masked "
+            "sample": f"{workload} workload: float64 gate on all of V (cost charged pro rata) + top-w and masked "
                       f"attention forward on the first {n_rows} query rows ({share * 100:.1f}% of kept pairs)",
             "seconds": round(secs, 3)}
 
@@ -683,9 +825,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-legs", action="store_true", help="skip the decode and training legs")
-    ap.add_argument("--legs", default="decode,train,chunk", help="comma-separated legs to run: decode, train, chunk")
+    ap.add_argument("--legs", default="long,decode,train,chunk",
+                    help="comma-separated legs to run: long, decode, train, chunk")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--clock-soak", type=float, default=1.5,
+                    help="seconds of untimed replays of the step, clock-sampled, before the timed region")
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)

@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DMA_ABI_VERSION 1
+#define DMA_ABI_VERSION 2
 
 /* Query rows per block of the mask encoding and of the attention kernels. */
 #define DMA_BLOCK_Q 128
@@ -90,15 +90,30 @@ typedef enum {
  *   w      window of the top-w selection, w >= 1 (w >= N keeps every causal key)
  *   scale  multiplier of q k^T; a value <= 0 selects 1/sqrt(d)
  *   dtype  a dma_dtype_t
+ *   flags  0, or DMA_FLAG_FORWARD_ONLY: a problem whose forward is not followed by a backward (inference
+ *          prefill): dma_attn_fwd then keeps nothing for a backward in the workspace (see dma_attn_fwd)
+ *          and dma_attn_bwd returns DMA_ERR_UNSUPPORTED.  Other bits are reserved (DMA_ERR_INVALID_ARG).
+ *   w_heads  NULL (every head selects with window w), or a device array of H int32 windows, one per
+ *          query head ("adaptive window sizing", section "Future Directions" of the page: the
+ *          window adapted per head, here supplied by the caller): head h selects with window
+ *          w_heads[h].  The kernels clamp each value to [1, w], so w must be the largest of them: it
+ *          sizes the workspace.  Every row of head h then keeps min(t+1, w_heads[h]) keys; the mask
+ *          encoding, the lists and the attention are otherwise unchanged.  The array is read on the
+ *          device by dma_topk_mask, dma_topk_append and the decode attention, and must hold the
+ *          same values for every call of one problem.
  *
  * Limits of this implementation (DMA_ERR_UNSUPPORTED beyond them): prefill/training
  * N <= 16384; decode N <= 1<<24 and min(w, N) <= 4096 * d; B*H <= 65535; d in {64, 128};
  * dma_gate, dma_gate_bwd and dma_gate_bwd_noalloc: H <= 64.
  */
+#define DMA_FLAG_FORWARD_ONLY 1
+
 typedef struct {
   int32_t B, H, Hkv, N, Nq, d, w;
   float scale;
   int32_t dtype;
+  int32_t flags;
+  const int32_t* w_heads;
 } dma_params_t;
 
 /*
@@ -116,7 +131,10 @@ typedef struct {
  *               by every row of the block (j <= t0 and e_j >= t1), then the partial ones (at
  *               most 2*DMA_BLOCK_Q); each group in ascending key order.  Entries past n_live
  *               are unspecified.
- *   off_sel     decode only: int32 [B, H, sel_len] selected keys of the query, ascending.
+ *   off_sel     decode only: int32 [B, H, sel_len] selected keys of the query, ascending:
+ *               sel_len = min(w, N), every row full; with w_heads, sel_len = w and row (b, h)
+ *               holds min(w_heads[h], N) keys (the rest unspecified), so that the row stride
+ *               stays the same as keys are appended.
  *   the rest    internal scratch.
  */
 typedef struct {
@@ -208,6 +226,9 @@ dma_status_t dma_gate_append(const dma_params_t* p, const void* V, const void* D
  *          and e_j from the per-entry copies dma_topk_mask stored with the lists, so a delta
  *          changed after dma_topk_mask is not seen there: run dma_topk_mask again.
  *   O      [B, H, Nq, d] dtype out;  LSE [B, H, Nq] float32 out
+ * With bfloat16 storage and Nq == N (a problem the backward can take) the call also keeps, in the
+ * workspace, the low-order part of every output, O - bf16(O), rounded to bfloat16, which
+ * dma_attn_bwd reads back; DMA_FLAG_FORWARD_ONLY skips it.
  */
 dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, const void* V,
                           const float* delta, const int32_t* evict, void* workspace,
@@ -215,7 +236,9 @@ dma_status_t dma_attn_fwd(const dma_params_t* p, const void* Q, const void* K, c
 
 /*
  * Masked attention backward (prefill/training only), selection held constant.
- *   O, LSE from dma_attn_fwd; dO [B, H, N, d] dtype.
+ *   O, LSE from dma_attn_fwd, on the same workspace: with bfloat16 storage the row sums
+ *   D_t = sum_c dO_tc O_tc use O plus the low-order part the forward kept there, so that D carries
+ *   O to about 16 significant bits rather than bfloat16's 8; dO [B, H, N, d] dtype.
  *   dQ [B, H, N, d], dK, dV [B, Hkv, N, d] dtype out (dK, dV summed over the query heads of
  *   each group);  d_delta [B, H, N] float32 out (sum over queries of dS_tj).
  */

@@ -55,6 +55,9 @@ __all__ = [
     "decode_select",
     "decode_select_append",
     "decode_attn",
+    "head_windows",
+    "topw_eviction_heads",
+    "decode_select_heads",
 ]
 
 
@@ -421,3 +424,37 @@ def decode_attn(q, K, V, delta, sel, scale=None):
             o[b, h] = (p / l) @ vv
             lse[b, h] = m + math.log(l)
     return o, lse
+
+
+# ----------------------------------------------------------------------------
+# Per-head windows ("Future Directions": adaptive window sizing; the window of
+# each head is supplied, the pages give no rule for choosing it)
+# ----------------------------------------------------------------------------
+
+def head_windows(w_heads, w: int) -> np.ndarray:
+    """The window each head selects with: w_heads[h] clamped to [1, w] (the
+    largest window w bounds every head's)."""
+    return np.clip(np.asarray(w_heads, dtype=np.int64), 1, w)
+
+
+def topw_eviction_heads(delta: np.ndarray, w_heads, w: int) -> np.ndarray:
+    """Eviction indices [B, H, N] when head h keeps the best min(t+1, W_h) keys
+    of every prefix, W = head_windows(w_heads, w): the m_t equation applied to
+    each head with its own window (the mask is per head, "a unique mask per
+    attention head")."""
+    B, H, N = delta.shape
+    W = head_windows(w_heads, w)
+    out = np.empty((B, H, N), dtype=np.int64)
+    for b in range(B):
+        for h in range(H):
+            out[b, h] = topw_eviction(delta[b, h], int(W[h]))
+    return out
+
+
+def decode_select_heads(delta: np.ndarray, w_heads, w: int) -> list:
+    """Decode selection with per-head windows: a list over (b, h) in row-major
+    order of the ascending selected keys of the query at position L-1 (row
+    (b, h) holds min(L, W_h) keys)."""
+    B, H, L = delta.shape
+    W = head_windows(w_heads, w)
+    return [decode_select(delta[b:b + 1, h:h + 1], int(W[h]))[0, 0] for b in range(B) for h in range(H)]

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported_and_bound():
 
 
 def test_abi_version_and_status_strings():
-    assert dma.abi_version() == 1
+    assert dma.abi_version() == 2
     lib = dma.load()
     for code in range(6):
         s = lib.dma_status_string(code).decode()
@@ -71,6 +71,29 @@ def test_params_validation(kw, expect):
     p = dma.make_params(**kw)
     st, _ = _ws_size(p)
     assert st == expect
+
+
+def test_misaligned_head_windows_pointer():
+    p = dma.make_params(1, 2, 1, 256, 64, 64, w_heads=(1 << 20) + 4)
+    assert _ws_size(p)[0] == INVALID
+    p = dma.make_params(1, 2, 1, 256, 64, 64, w_heads=1 << 20)
+    assert _ws_size(p)[0] == OK
+
+
+def test_decode_selection_stride_with_head_windows():
+    # without per-head windows the rows hold min(w, N) keys; with them the stride is w whatever N is
+    assert dma.workspace_layout(dma.make_params(1, 2, 1, 100, 64, 300, Nq=1)).sel_len == 100
+    assert dma.workspace_layout(dma.make_params(1, 2, 1, 100, 64, 300, Nq=1, w_heads=1 << 20)).sel_len == 300
+
+
+def test_flags():
+    p = dma.make_params(1, 2, 1, 256, 64, 64)
+    p.flags = 2
+    assert _ws_size(p)[0] == INVALID
+    # a forward-only problem keeps nothing for a backward: a smaller workspace
+    full = dma.workspace_size(dma.make_params(1, 16, 8, 4096, 128, 1024))
+    fwd = dma.workspace_size(dma.make_params(1, 16, 8, 4096, 128, 1024, forward_only=True))
+    assert full - fwd >= 16 * 4096 * 128 * 2
 
 
 def test_bad_dtype_and_scale():
@@ -139,6 +162,9 @@ assert lib.dma_attn_bwd(pp, *args_bad) == INVALID
 assert lib.dma_gate_bwd(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == INVALID
 # gate_bwd_noalloc(p, V, Delta, A, x_save, delta, d_delta, dDelta, dA, dV_gate, stream)
 assert lib.dma_gate_bwd_noalloc(pp, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, None) == INVALID
+pf = dma.make_params(1, 2, 1, 256, 64, 64, forward_only=True)   # forward-only: no backward
+args = [FAKE] * 6 + [need_of(pf)] + [FAKE] * 7 + [None]
+assert lib.dma_attn_bwd(ctypes.byref(pf), *args) == UNSUPPORTED
 pc = dma.make_params(1, 2, 1, 256, 64, 64, Nq=100)   # chunked prefill: no backward
 args = [FAKE] * 6 + [need_of(pc)] + [FAKE] * 7 + [None]
 assert lib.dma_attn_bwd(ctypes.byref(pc), *args) == UNSUPPORTED

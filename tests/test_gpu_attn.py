@@ -99,16 +99,42 @@ def test_attn_fwd_full(case):
     assert_close(to_np(O), O_ref, "O")
 
 
-@pytest.mark.parametrize("name", ["long", "train"])
-def test_attn_fwd_sampled_rows_full_size(name):
-    """Full-size workloads in the benchmark's launch configuration; the oracle
-    recomputes a seeded sample of query rows (every block edge included)."""
-    wl = get(name)
+def test_attn_fwd_forward_only_flag_same_outputs():
+    """DMA_FLAG_FORWARD_ONLY changes what the forward keeps for a backward, never its outputs:
+    O and LSE bit for bit equal to those of the same problem without the flag."""
+    wl = get("prefill").with_(H=4, Hkv=2, N=1500, seed=27)
     dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl)
     O, LSE = _fwd(dma, torch, wl, p, ws, dev)
-    rng = np.random.default_rng(99)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, wl.N - 129, wl.N - 1],
-                                     rng.choice(wl.N, size=58, replace=False)]))
+    p1 = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype=wl.dtype, forward_only=True)
+    ws1 = dma.alloc_workspace(p1)
+    dma.topk_mask(p1, dev["delta"], dev["evict"], ws1)
+    O1, LSE1 = _fwd(dma, torch, wl, p1, ws1, dev)
+    assert torch.equal(O.view(torch.int16), O1.view(torch.int16)) and torch.equal(LSE, LSE1)
+    O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, gemm_dtype=np.float32)
+    assert_close(to_np(O1), O_ref, "O")
+
+
+def _sample_rows(N, n, seed):
+    """A seeded sample of n query rows that always holds both edges of every pair
+    of 128-row blocks near the start and the end (row 0, the first block edges,
+    the last full pair and the ragged tail)."""
+    rng = np.random.default_rng(seed)
+    edges = np.array([0, 1, 127, 128, 255, 256, N - 257, N - 256, N - 129, N - 128, N - 1])
+    edges = edges[(edges >= 0) & (edges < N)]
+    rest = rng.choice(np.setdiff1d(np.arange(N), edges), size=max(0, n - edges.size), replace=False)
+    return np.unique(np.concatenate([edges, rest]))
+
+
+def test_attn_fwd_long_sampled_rows_full_size():
+    """The long workload at full size in the benchmark's launch configuration;
+    the oracle recomputes a seeded sample of 2048 query rows of every head (the
+    same rows in every head; block edges and the ragged end included).  The
+    training workload's forward is checked in full with its backward below."""
+    wl = get("long")
+    dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl)
+    O, LSE = _fwd(dma, torch, wl, p, ws, dev)
+    rows = _sample_rows(wl.N, 2048, 99)
+    assert rows.size == 2048
     O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, rows=rows, gemm_dtype=np.float32)
     assert_close(to_np(LSE)[:, :, rows], L_ref[:, :, rows], "LSE")
     assert_close(to_np(O)[:, :, rows], O_ref[:, :, rows], "O")
@@ -150,22 +176,25 @@ def test_attn_bwd_full(case):
         assert_close(to_np(g), ref, name)
 
 
-def test_attn_bwd_train_full_size_one_group():
-    """The training workload at full size on the GPU; the oracle checks every
-    gradient of batch 0, KV group 0 (its two query heads), dense."""
+def test_attn_bwd_train_full_size_every_head():
+    """The training workload at full size on the GPU (the benchmark's launch
+    configuration): O and LSE of every query row, then every gradient of every
+    head, batch row and KV group against the oracle's dense analytic backward
+    (float32 GEMMs, float64 row reductions), element by element: dQ, dK, dV and
+    d_delta in full."""
     wl = get("train")
     dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl, with_dO=True)
     O, LSE = _fwd(dma, torch, wl, p, ws, dev)
     dQ, dK, dV, dd = _bwd(dma, torch, wl, p, ws, dev, O, LSE)
-    G = wl.G
-    sl_q = (slice(0, 1), slice(0, G))
-    sl_k = (slice(0, 1), slice(0, 1))
-    r = oracle.attn_bwd(I.Q[sl_q], I.K[sl_k], I.V[sl_k], d32[sl_q].astype(np.float64), e_ref[sl_q], I.dO[sl_q],
-                        gemm_dtype=np.float32)
-    assert_close(to_np(dQ[sl_q]), r[0], "dQ")
-    assert_close(to_np(dK[sl_k]), r[1], "dK")
-    assert_close(to_np(dV[sl_k]), r[2], "dV")
-    assert_close(to_np(dd[sl_q]), r[3], "d_delta")
+    got = [to_np(t) for t in (dQ, dK, dV, dd)]
+    del dQ, dK, dV, dd
+    O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, gemm_dtype=np.float32)
+    assert_close(to_np(LSE), L_ref, "LSE")
+    assert_close(to_np(O), O_ref, "O")
+    del O_ref, L_ref
+    r = oracle.attn_bwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, I.dO, gemm_dtype=np.float32)
+    for name, g, ref in zip(("dQ", "dK", "dV", "d_delta"), got, r):
+        assert_close(g, ref, name)
 
 
 # ---------------------------------------------------------------- gate backward

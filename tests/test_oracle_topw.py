@@ -104,3 +104,52 @@ def test_live_keys_per_block_against_mask(N, w):
             # the live set never exceeds w + Bq keys, the partial keys never 2 Bq
             assert full.size + partial.size <= w + Bq
             assert partial.size <= 2 * Bq
+
+
+# ---------------------------------------------------------------- per-head windows
+
+def test_head_windows_clamp():
+    np.testing.assert_array_equal(oracle.head_windows([0, 1, 5, 9, 100], 9), [1, 1, 5, 9, 9])
+
+
+@pytest.mark.parametrize("kind,levels", [("uniform", 0), ("levels", 4), ("constant", 0)])
+def test_eviction_heads_equals_brute_force_per_head(kind, levels):
+    """Each head's mask is the brute-force selection with that head's own window
+    (windows below, at and above the row length; one above the largest window is
+    clamped to it)."""
+    N, w = 37, 30
+    w_heads = [1, 4, 13, 30, 45]
+    d = make_delta((2, len(w_heads), N), seed=91, kind=kind, levels=levels)
+    e = oracle.topw_eviction_heads(d, w_heads, w)
+    eff = [1, 4, 13, 30, 30]
+    for b in range(2):
+        for h, wh in enumerate(eff):
+            M = oracle.topw_sets_bruteforce(d[b, h], wh)
+            np.testing.assert_array_equal(oracle.mask_from_eviction(e[b, h]), M)
+            assert (M.sum(axis=1) == np.minimum(np.arange(N) + 1, wh)).all()
+
+
+def test_eviction_heads_increasing_is_a_window_per_head():
+    """Strictly increasing delta: head h attends to the sliding window of its
+    own width W_h, [t - W_h + 1, t]."""
+    N = 50
+    w_heads = [3, 11, 50]
+    d = make_delta((1, 3, N), seed=0, kind="increasing")
+    e = oracle.topw_eviction_heads(d, w_heads, 50)
+    for h, wh in enumerate(w_heads):
+        expect = np.minimum(np.arange(N) + wh, N)
+        np.testing.assert_array_equal(e[0, h], expect)
+
+
+def test_decode_select_heads_by_sorting():
+    """Row (b, h) holds the min(L, W_h) best keys by (delta desc, index asc), ascending."""
+    rng = np.random.default_rng(5)
+    B, H, L, w = 2, 3, 40, 25
+    d = np.round(rng.random((B, H, L)).astype(np.float32) * 8) / 8   # many ties
+    w_heads = [25, 2, 60]
+    rows = oracle.decode_select_heads(d, w_heads, w)
+    eff = [25, 2, 25]
+    for b in range(B):
+        for h in range(H):
+            order = sorted(range(L), key=lambda j: (-float(d[b, h, j]), j))
+            np.testing.assert_array_equal(rows[b * H + h], sorted(order[:min(L, eff[h])]))

@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import ctypes
 
-from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DmaError, DmaParams, DmaWsLayout, LIB_PATH, check,
+from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DMA_FLAG_FORWARD_ONLY, DmaError, DmaParams, DmaWsLayout, LIB_PATH, check,
                    exported_names, load)
 
 __all__ = [
@@ -26,11 +26,20 @@ __all__ = [
 ]
 
 
-def make_params(B, H, Hkv, N, d, w, Nq=None, scale=0.0, dtype="bf16") -> DmaParams:
-    """dma_params_t for a problem (Nq defaults to N; Nq=1 is decode)."""
+def make_params(B, H, Hkv, N, d, w, Nq=None, scale=0.0, dtype="bf16", w_heads=None,
+                forward_only=False) -> DmaParams:
+    """dma_params_t for a problem (Nq defaults to N; Nq=1 is decode).
+
+    forward_only: no backward follows (DMA_FLAG_FORWARD_ONLY): the forward keeps
+    nothing for it in the workspace.
+
+    w_heads: None, or per-head windows as a device int32 tensor of H values (or its
+    device address); w must then be the largest of them.  The caller keeps the
+    tensor alive for as long as the parameters are used."""
     dt = {"bf16": DMA_BF16, "f32": DMA_F32}[dtype] if isinstance(dtype, str) else int(dtype)
     return DmaParams(B=B, H=H, Hkv=Hkv, N=N, Nq=N if Nq is None else Nq, d=d, w=w,
-                     scale=float(scale), dtype=dt)
+                     scale=float(scale), dtype=dt, flags=DMA_FLAG_FORWARD_ONLY if forward_only else 0,
+                     w_heads=_ptr(w_heads))
 
 
 def abi_version() -> int:

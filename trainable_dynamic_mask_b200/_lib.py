@@ -21,13 +21,15 @@ STATUS_NAMES = {0: "DMA_OK", 1: "DMA_ERR_INVALID_ARG", 2: "DMA_ERR_UNSUPPORTED",
                 3: "DMA_ERR_WORKSPACE", 4: "DMA_ERR_CUDA", 5: "DMA_ERR_TIMEOUT"}
 DMA_BF16 = 0
 DMA_F32 = 1
+DMA_FLAG_FORWARD_ONLY = 1
 BLOCK_Q = 128
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class DmaParams(ctypes.Structure):
     _fields_ = [("B", c_i32), ("H", c_i32), ("Hkv", c_i32), ("N", c_i32), ("Nq", c_i32),
-                ("d", c_i32), ("w", c_i32), ("scale", c_f32), ("dtype", c_i32)]
+                ("d", c_i32), ("w", c_i32), ("scale", c_f32), ("dtype", c_i32), ("flags", c_i32),
+                ("w_heads", c_vp)]
 
 
 class DmaWsLayout(ctypes.Structure):

@@ -136,11 +136,15 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
   if (p->dtype != DMA_BF16 && p->dtype != DMA_F32) return DMA_ERR_INVALID_ARG;
   if (p->Nq > p->N) return DMA_ERR_INVALID_ARG;
   if (!(p->scale == p->scale) || isinf(p->scale)) return DMA_ERR_INVALID_ARG;
+  if (p->w_heads != nullptr && (reinterpret_cast<uintptr_t>(p->w_heads) & 15u) != 0) return DMA_ERR_INVALID_ARG;
+  if ((p->flags & ~DMA_FLAG_FORWARD_ONLY) != 0) return DMA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return DMA_ERR_UNSUPPORTED;
   if ((int64_t)p->B * p->H > 65535) return DMA_ERR_UNSUPPORTED;
   Plan& R = *P;
   memset(&R, 0, sizeof(R));
   R.B = p->B; R.H = p->H; R.Hkv = p->Hkv; R.N = p->N; R.Nq = p->Nq; R.d = p->d; R.w = p->w;
+  R.w_heads = p->w_heads;
+  R.fwd_only = (p->flags & DMA_FLAG_FORWARD_ONLY) != 0;
   R.G = p->H / p->Hkv;
   R.scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->d);
   R.bf16 = p->dtype == DMA_BF16;
@@ -161,7 +165,9 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.pair_cap = (int)(pcap < ncap ? pcap : ncap);
   }
   R.n_pairs = (R.N + kPairQ - 1) / kPairQ;
-  R.sel_len = minwn;
+  // with per-head windows the selection rows keep the stride w whatever N is, so that an appended
+  // key never moves a row (each row holds min(w_h, N) keys)
+  R.sel_len = R.w_heads != nullptr ? R.w : minwn;
   R.n_split = (R.sel_len + kDecodeSplit - 1) / kDecodeSplit;
   // decode combines its splits' (m, l) in shared memory, within kDecodeSplit * d * 2 bytes
   if (R.decode && (size_t)R.n_split * 2 * sizeof(float) > (size_t)kDecodeSplit * R.d * 2) return DMA_ERR_UNSUPPORTED;
@@ -186,6 +192,8 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     R.off_fml = take((size_t)R.sched.n_slots * 2 * 2 * kBlockQ * sizeof(float));
     R.off_fcnt = take((BH * R.n_pairs * 4 + 2) * sizeof(int32_t));   // + the forward's unit counters
     R.off_rowD = take(BH * R.Nq * sizeof(float));
+    // the forward keeps the low-order bf16 part of O for the backward (training: every position a query)
+    if (R.bf16 && R.q0 == 0 && !R.fwd_only) R.off_olo = take(BH * R.n_blocks * (size_t)kBlockQ * R.d * 2);
     {
       const size_t n_slots = BH * ((R.N + 1023) / 1024) * 8;   // windows of 1024 keys, tiles of 128
       R.off_dkv_perm = take(BH * R.N * sizeof(int32_t));
@@ -344,7 +352,7 @@ dma_status_t dma_attn_bwd(const dma_params_t* p, const void* Q, const void* K, c
   Plan P;
   dma_status_t st = make_plan(p, &P);
   if (st != DMA_OK) return st;
-  if (P.decode || P.q0 != 0) return DMA_ERR_UNSUPPORTED;   // training: every position is a query
+  if (P.decode || P.q0 != 0 || P.fwd_only) return DMA_ERR_UNSUPPORTED;   // training: every position a query
   if (!ok_ptr(Q) || !ok_ptr(K) || !ok_ptr(V) || !ok_ptr(delta) || !ok_ptr(evict) || !ok_ptr(O) ||
       !ok_ptr(LSE) || !ok_ptr(dO) || !ok_ptr(dQ) || !ok_ptr(dK) || !ok_ptr(dV) || !ok_ptr(d_delta))
     return DMA_ERR_INVALID_ARG;

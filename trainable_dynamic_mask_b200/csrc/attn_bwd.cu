@@ -19,52 +19,61 @@ namespace dma {
 namespace {
 
 // ---------------------------------------------------------------- D = rowsum(dO * O)
-// One warp per kRowdotRows rows; each lane reads 4 consecutive elements of O and of dO per row (8- or
-// 16-byte loads), the loads of all the warp's rows issued before the sums.
-DMA_DEVINL void load4_f32(const uint16_t* p, float (&v)[4]) {
-  const uint2 w = *reinterpret_cast<const uint2*>(p);
-  v[0] = __uint_as_float(w.x << 16);
-  v[1] = __uint_as_float(w.x & 0xffff0000u);
-  v[2] = __uint_as_float(w.y << 16);
-  v[3] = __uint_as_float(w.y & 0xffff0000u);
-}
-DMA_DEVINL void load4_f32(const float* p, float (&v)[4]) {
-  const float4 w = *reinterpret_cast<const float4*>(p);
-  v[0] = w.x;
-  v[1] = w.y;
-  v[2] = w.z;
-  v[3] = w.w;
-}
-
-constexpr int kRowdotRows = 4;   // rows per warp, loaded together
-
-template <typename OT>
-__global__ void bwd_rowdot_kernel(const OT* __restrict__ O, const uint16_t* __restrict__ dO,
-                                  float* __restrict__ Drow, size_t rows, int D) {
-  const size_t r0 = ((size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * kRowdotRows;
-  const int lane = threadIdx.x & 31;
-  if (r0 >= rows) return;
-  float acc[kRowdotRows];
-  for (int c = lane * 4; c < D; c += 128) {
-    float o[kRowdotRows][4], g[kRowdotRows][4];
+// One CTA per 128-row block of one (b, h), one thread per row: the thread walks its row in groups of
+// 8 columns (16-byte loads of O and dO; the row's 128-byte lines stay in L1 across the groups), four
+// groups' loads in flight together.  With Olo (bf16 storage) the row of O is O + Olo, the output plus
+// the low-order part the forward kept in its blocked layout [128-row block][D / 8][128 rows][8], read
+// by the 32 lanes of a warp as 512 contiguous bytes: D then carries O to about 16 significant bits.
+// D_t weighs every dS of row t; with O rounded to bf16 its error alone moved the column sums of dS
+// (d delta) of keys that the first rows select (large P and large |O|) by more than the parity
+// tolerance.
+DMA_DEVINL void load8_f32(const uint16_t* p, float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int k = 0; k < kRowdotRows; ++k) {
-      const size_t r = r0 + k < rows ? r0 + k : r0;
-      load4_f32(O + r * D + c, o[k]);
-      load4_f32(dO + r * D + c, g[k]);
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(u[k] << 16);
+    v[2 * k + 1] = __uint_as_float(u[k] & 0xffff0000u);
+  }
+}
+DMA_DEVINL void load8_f32(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+constexpr int kRowdotBlock = DMA_BLOCK_Q;   // rows per CTA (one per thread)
+constexpr int kRowdotBatch = 4;             // column groups loaded together
+
+template <int D, typename OT>
+__global__ void __launch_bounds__(kRowdotBlock)
+bwd_rowdot_kernel(const OT* __restrict__ O, const uint16_t* __restrict__ Olo, const uint16_t* __restrict__ dO,
+                  float* __restrict__ Drow, int N) {
+  constexpr int NG = D / 8;
+  const int blk = blockIdx.x, bh = blockIdx.y, r = threadIdx.x;
+  const int t = blk * kRowdotBlock + r;
+  if (t >= N) return;
+  const size_t row = (size_t)bh * N + t;
+  const uint16_t* lo = Olo != nullptr
+                           ? Olo + ((size_t)bh * gridDim.x + blk) * kRowdotBlock * D + (size_t)r * 8
+                           : nullptr;
+  float acc = 0.f;
+#pragma unroll
+  for (int g0 = 0; g0 < NG; g0 += kRowdotBatch) {
+    float o[kRowdotBatch][8], g[kRowdotBatch][8], l[kRowdotBatch][8];
+#pragma unroll
+    for (int k = 0; k < kRowdotBatch; ++k) {
+      load8_f32(O + row * D + (g0 + k) * 8, o[k]);
+      load8_f32(dO + row * D + (g0 + k) * 8, g[k]);
+      if (lo != nullptr) load8_f32(lo + (size_t)(g0 + k) * kRowdotBlock * 8, l[k]);
     }
 #pragma unroll
-    for (int k = 0; k < kRowdotRows; ++k)
-      acc[k] = fmaf(o[k][0], g[k][0], fmaf(o[k][1], g[k][1], fmaf(o[k][2], g[k][2],
-                    fmaf(o[k][3], g[k][3], c == lane * 4 ? 0.f : acc[k]))));
-  }
+    for (int k = 0; k < kRowdotBatch; ++k)
 #pragma unroll
-  for (int k = 0; k < kRowdotRows; ++k) {
-    float v = lane * 4 < D ? acc[k] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && r0 + k < rows) Drow[r0 + k] = v;
+      for (int u = 0; u < 8; ++u) acc = fmaf(lo != nullptr ? o[k][u] + l[k][u] : o[k][u], g[k][u], acc);
   }
+  Drow[row] = acc;
 }
 
 template <int D, typename OutT>
@@ -73,10 +82,9 @@ cudaError_t launch_bwd_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
                          const float* LSE, const uint16_t* dO, void* dQ, void* dK, void* dV,
                          float* d_delta, cudaStream_t s) {
   float* Drow = ws_ptr<float>(ws, P.off_rowD);
-  const size_t rows = (size_t)P.B * P.H * P.N;
-  const size_t per_block = 8 * kRowdotRows;
-  bwd_rowdot_kernel<OutT><<<(unsigned)((rows + per_block - 1) / per_block), 256, 0, s>>>((const OutT*)O, dO, Drow,
-                                                                                       rows, D);
+  const uint16_t* Olo = P.off_olo ? ws_ptr<uint16_t>(ws, P.off_olo) : nullptr;
+  bwd_rowdot_kernel<D, OutT><<<dim3(P.n_blocks, P.B * P.H), kRowdotBlock, 0, s>>>((const OutT*)O, Olo, dO, Drow,
+                                                                                  P.N);
   {
     cudaError_t e = launch_bwd_dq_tc(P, Q, K, V, dO, delta, evict, ws, LSE, Drow, dQ, s);
     if (e != cudaSuccess) return e;

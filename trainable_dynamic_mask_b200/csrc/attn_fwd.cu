@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kDecThreads)
 decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
                     const uint16_t* __restrict__ V, const float* __restrict__ delta,
                     const int32_t* __restrict__ sel, float* __restrict__ part, int H, int G, int N,
-                    int sel_len, int n_split, float scale_log2) {
+                    int sel_len, int n_split, float scale_log2, int w, const int32_t* __restrict__ w_heads) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
   constexpr int NG = kDecThreads / CH;      // key groups of the weighted V sum
   static_assert(kDecodeSplit == kDecThreads, "one key per thread");
@@ -49,7 +49,10 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
   const uint16_t* Kg = K + (size_t)(b * Hkv + g) * N * D;
   const uint16_t* Vg = V + (size_t)(b * Hkv + g) * N * D;
   const int k0 = s * kDecodeSplit;
-  const int nk = min(kDecodeSplit, sel_len - k0);
+  // the row holds min(window, N) selected keys (sel_len is the row stride; with per-head windows a
+  // row may hold fewer, and splits past its end reduce nothing: m = -inf, l = 0)
+  const int n_row = min(row_window(w_heads, bh, H, w), N);
+  const int nk = min(kDecodeSplit, n_row - k0);
   const int j = tid < nk ? sel[(size_t)bh * sel_len + k0 + tid] : -1;
   idx[tid] = j;
   const float dl = j >= 0 ? delta[(size_t)bh * N + j] * kLog2e : 0.f;
@@ -196,7 +199,7 @@ cudaError_t launch_dec_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
   }
   decode_split_kernel<D><<<dim3(P.n_split, P.B * P.H), kDecThreads, decode_smem_bytes<D>(), s>>>(
       Q, K, V, delta, ws_ptr<int32_t>(ws, P.off_sel), part, P.H, P.G, P.N, P.sel_len, P.n_split,
-      P.scale * kLog2e);
+      P.scale * kLog2e, P.w, P.w_heads);
   decode_combine_kernel<D, OutT><<<P.B * P.H, D, 2 * P.n_split * sizeof(float), s>>>(part, (OutT*)O, LSE,
                                                                                       P.n_split);
   return cudaGetLastError();

@@ -18,15 +18,22 @@
 //   warps 0-3  softmax of query half 0, warps 4-7 softmax of half 1: thread r owns query row r of
 //              its half = TMEM lane r.  It reads its S row from TMEM, applies scale, +delta_j and the
 //              mask j <= t < e_j (tiles of full keys skip the test), keeps the running max and sum,
-//              writes P (bf16) over S in TMEM, and rescales its O row only when the running max
-//              grows by more than 2^8 (the stale max otherwise stays the reference).  A quarter of
-//              the exponentials run as a polynomial on the FMA pipe to offload the MUFU pipe;
+//              writes P (bf16) over S in TMEM, and rescales its O row whenever the running max
+//              grows.  The reference of P is thus always the exact running max, so P <= 1 and the
+//              key that holds the row's maximum enters with P = 1 exactly: a stale reference (P up
+//              to 2^k) rounds the dominant weight to bf16 too, and in rows dominated by a few large
+//              value rows (scaled keys of the long workload) that rounding alone moved outputs by
+//              more than the parity tolerance.  A quarter of the exponentials run as a polynomial
+//              on the FMA pipe to offload the MUFU pipe;
 //   warp 8     allocates TMEM; one thread issues the MMAs: S_h = Q_h K^T (operands in shared
 //              memory) and O_h += P_h V (P_h from TMEM, V from shared memory);
 //   warps 9-11 gather V rows, warps 12-15 gather Q and K rows, with TMA tile::gather4 (128-byte
 //              swizzled, the layout the MMA reads).  One warp's TMA issue rate caps its gather
 //              throughput, so seven warps issue.
-// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D); P_h aliases S_h.
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [384,384+D); P_h aliases S_h.  The MMAs
+// of one thread execute in issue order, so S_h of tile i + 1 is issued right behind the PV of tile i
+// that reads P_h (no wait for that PV to complete): the tensor pipe holds both while the softmax of
+// the other half runs.
 // Stages: Q 1 (both halves), K 2, V 2.  Tile metadata (delta_j log2(e), j, e_j - j) is read by
 // the softmax threads straight from the list, one entry per thread, through a shared buffer.
 // Every wait is bounded (tc::mbar_wait) and reports a timeout through the workspace status word;
@@ -51,7 +58,6 @@ constexpr int kKWarp0 = 12;                 // Q/K producers: warps 12-15, row g
 constexpr int kRegsSoftmax = 208, kRegsOther = 48;
 constexpr int kTcBK = 128;                  // keys per tile
 constexpr int kKStages = 2, kVStages = 2;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr int kPolyEvery = 4;               // one pair in kPolyEvery takes the polynomial exp2
 constexpr int kSchedRing = 4;               // units published ahead by the scheduling thread
 constexpr int kSchedConsumers = 15;         // warps that read each published unit (all but the scheduler's)
@@ -193,7 +199,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
                    const __grid_constant__ CUtensorMap vmap, const __grid_constant__ FwdSchedule sched,
                    const int32_t* __restrict__ pcounts, const int32_t* __restrict__ plists,
                    const int32_t* __restrict__ plen, const float* __restrict__ pdl, OutT* __restrict__ O,
-                   float* __restrict__ LSE, float* __restrict__ fpart, float* __restrict__ fml,
+                   float* __restrict__ LSE, uint16_t* __restrict__ Olo, float* __restrict__ fpart,
+                   float* __restrict__ fml,
                    int32_t* __restrict__ fcnt, int32_t* __restrict__ sched_ctr, int32_t* __restrict__ status, int H,
                    int G, int N, int n_pairs,
                    int pair_cap, float scale_log2, int q0) {
@@ -348,16 +355,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
           const int n_tiles = te - tb;
           if (n_tiles == 0) continue;
           if (!(ok = tc::mbar_wait(&bar.q_full, n_done & 1, abort_flag, status, kErrTimeoutQ))) break;
-          // first K tile: both halves
+          // first K tile: both halves.  S_h overwrites P_h of the previous item's last tile, which that
+          // item's last PV (issued earlier by this thread) reads: tcgen05.mma operations issued by one
+          // thread execute in issue order, so the write cannot overtake the read and needs no wait.
           if (!(ok = tc::mbar_wait(&bar.k_full[kc % 2], (kc / 2) & 1, abort_flag, status, kErrTimeoutK))) break;
           tc::fence_after();
-          for (int half = 0; half < 2 && ok; ++half) {
-            // S_h / P_h of the previous item is free once its last PV has completed
-            if (tcount > 0)
-              ok = tc::mbar_wait(&bar.pv_done[half], (tcount - 1) & 1, abort_flag, status, kErrTimeoutPV);
-            if (ok) issue_qk<D>(tmem, half, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[half]);
-          }
-          if (!ok) break;
+          for (int half = 0; half < 2; ++half)
+            issue_qk<D>(tmem, half, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[half]);
           tc::commit(&bar.k_empty[kc % 2]);
           ++kc;
           if (n_tiles == 1) tc::commit(&bar.q_empty);
@@ -371,9 +375,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             issue_pv<D>(tmem, 0, dv0 + (uint64_t)((vs * S::kTile) >> 4), i == 0, &bar.pv_done[0]);
             const bool more = i + 1 < n_tiles;
             if (more) {
-              ok = tc::mbar_wait(&bar.k_full[kc % 2], (kc / 2) & 1, abort_flag, status, kErrTimeoutK) &&
-                   tc::mbar_wait(&bar.pv_done[0], t & 1, abort_flag, status, kErrTimeoutPV);
-              if (!ok) break;
+              // S_0 of the next tile goes over P_0, which the PV just issued reads: in-order execution
+              // of this thread's MMAs orders the two (no wait for the PV to complete)
+              if (!(ok = tc::mbar_wait(&bar.k_full[kc % 2], (kc / 2) & 1, abort_flag, status, kErrTimeoutK))) break;
               tc::fence_after();
               issue_qk<D>(tmem, 0, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[0]);
             }
@@ -383,8 +387,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
             tc::commit(&bar.v_empty[vs]);
             ++vc;
             if (more) {
-              if (!(ok = tc::mbar_wait(&bar.pv_done[1], t & 1, abort_flag, status, kErrTimeoutPV))) break;
-              tc::fence_after();
               issue_qk<D>(tmem, 1, dq0, dk0 + (uint64_t)(((kc % 2) * S::kTile) >> 4), &bar.s_full[1]);
               tc::commit(&bar.k_empty[kc % 2]);
               ++kc;
@@ -500,7 +502,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         }
         float alpha = 1.f;
         bool rescale = false;
-        if (mt > m_used + kRescaleThreshold || (m_used == -INFINITY && mt != -INFINITY)) {
+        if (mt > m_used) {   // (also the first finite max: -inf < mt)
           alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
           m_used = mt;
           rescale = true;
@@ -534,14 +536,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
         // p_full).  O_h holds this item's tiles < i: their PV completed before S_h of tile i was
         // computed.  The whole warp rescales when any of its rows needs it (alpha = 1 for the others).
         if (i > 0 && __any_sync(0xffffffffu, rescale)) {
+          // the S row is dead: its registers take the whole O row, loaded with one wait
+          uint32_t (&orow)[kTcBK / 32][32] = sr;
+          static_assert(D <= kTcBK, "the O row reuses the S row's registers");
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tc::tmem_ld32(tO + c * 32, orow[c]);
+          tc::tmem_wait_ld();
+          const uint64_t a2 = f2(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            uint32_t orow[32];
-            tc::tmem_ld32(tO + c * 32, orow);
-            tc::tmem_wait_ld();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) orow[u] = __float_as_uint(__uint_as_float(orow[u]) * alpha);
-            tc::tmem_st32(tO + c * 32, orow);
+            for (int u = 0; u < 32; u += 2) {
+              float o0, o1;
+              f2_split(f2_mul(f2(__uint_as_float(orow[c][u]), __uint_as_float(orow[c][u + 1])), a2), o0, o1);
+              orow[c][u] = __float_as_uint(o0);
+              orow[c][u + 1] = __float_as_uint(o1);
+            }
+            tc::tmem_st32(tO + c * 32, orow[c]);
           }
         }
         float s0, s1, s2, s3;
@@ -565,6 +576,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
       }
       const bool valid = t >= q0 && t < N;   // a query row (rows of the first pair below q0 are not)
       OutT* orow = O + ((size_t)it.bh * Nq + (valid ? t - q0 : 0)) * D;
+      // low-order bf16 part of the row (O - bf16(O)), kept for the backward's D = rowsum(dO * O), in
+      // the blocked layout [b, h][128-row block][D / 8 column groups][128 rows][8]: this thread's row is
+      // row r of block 2 kp + h (kept only when every position is a query, q0 = 0)
+      uint16_t* lblk = Olo + ((size_t)it.bh * ((Nq + kBlockQ - 1) / kBlockQ) + it.kp * 2 + h) * kBlockQ * D;
+      const bool keep_lo = valid && Olo != nullptr;
       if (it.S == 1) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
@@ -576,6 +592,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 #pragma unroll
           for (int u2 = 0; u2 < 32; ++u2) of[u2] = __uint_as_float(ov[u2]) * inv;
           if (valid) store_row32(orow + c * 32, of);
+          if (keep_lo) store_row32_lo(lblk + (size_t)c * 4 * kBlockQ * 8, r, of);
         }
         if (valid) LSE[(size_t)it.bh * Nq + t - q0] = ((m_used == -INFINITY ? 0.f : m_used) + __log2f(l)) * kLn2;
       } else {
@@ -651,6 +668,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_consta
 #pragma unroll
             for (int u2 = 0; u2 < 32; ++u2) of[u2] *= inv;
             if (valid) store_row32(orow + c * 32, of);
+            if (keep_lo) store_row32_lo(lblk + (size_t)c * 4 * kBlockQ * 8, r, of);
           }
           if (valid) LSE[(size_t)it.bh * Nq + t - q0] = (Mb + __log2f(L)) * kLn2;
           group_sync(h);
@@ -696,7 +714,9 @@ cudaError_t launch_tc_t(const Plan& P, const uint16_t* Q, const uint16_t* K, con
   (void)evict;
   k<<<grid, kTcThreads, smem, s>>>(qm, km, vm, P.sched, ws_ptr<int32_t>(ws, P.off_pcounts),
                                    ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
-                                   ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE, ws_ptr<float>(ws, P.off_fpart),
+                                   ws_ptr<float>(ws, P.off_pdl), (OutT*)O, LSE,
+                                   P.off_olo ? ws_ptr<uint16_t>(ws, P.off_olo) : nullptr,
+                                   ws_ptr<float>(ws, P.off_fpart),
                                    ws_ptr<float>(ws, P.off_fml), ws_ptr<int32_t>(ws, P.off_fcnt),
                                    ws_ptr<int32_t>(ws, P.off_fcnt) + (size_t)P.B * P.H * P.n_pairs * 4,
                                    ws_ptr<int32_t>(ws, P.off_status), P.H, P.G, P.N, P.n_pairs, P.pair_cap,

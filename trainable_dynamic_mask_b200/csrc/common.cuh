@@ -43,6 +43,14 @@ DMA_DEVINL uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Window of selection row `row` (= b * H + h): w_heads[h] clamped to [1, w], or w when there are no
+// per-head windows.
+DMA_DEVINL int row_window(const int32_t* w_heads, int row, int H, int w) {
+  if (w_heads == nullptr) return w;
+  const int v = __ldg(w_heads + row % H);
+  return v < 1 ? 1 : (v > w ? w : v);
+}
+
 // ---------------------------------------------------------------- shared-memory access
 
 DMA_DEVINL uint32_t smem_u32(const void* p) {

@@ -39,16 +39,18 @@ struct FwdSchedule {
 // Resolved problem and workspace plan.
 struct Plan {
   int B, H, Hkv, N, Nq, d, w, G;
+  const int32_t* w_heads;   // per-head windows (device, [H]) or nullptr: every head uses w
   float scale;
   bool bf16;      // storage dtype is bf16 (else f32)
   bool decode;    // Nq == 1 and N > 1 ... the single query sits at position N-1
+  bool fwd_only;  // DMA_FLAG_FORWARD_ONLY: no backward follows the forward
   int q0;         // first query position, N - Nq: 0 (prefill), N - 1 (decode), else a chunk of a longer
                   // sequence (chunked prefill: the queries are the last Nq positions)
   int n_blocks;   // query blocks of kBlockQ rows (prefill)
   int list_cap;   // entries per block list
   int n_pairs;    // query blocks of kPairQ rows (attention forward work items)
   int pair_cap;   // entries per pair list (a multiple of 128; every list is padded to 128)
-  int sel_len;    // decode: min(w, N)
+  int sel_len;    // decode: row stride of the selection, min(w, N) (w with per-head windows)
   int n_split;    // decode: splits per (b, h)
   int n_slices;   // gate backward: position slices of kGateSlice
   // byte offsets in the workspace
@@ -56,6 +58,8 @@ struct Plan {
   size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
   size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
+  size_t off_olo;                      // bf16 prefill/training: O - bf16(O) as bf16, blocked
+                                       // [B, H][n_blocks][d / 8][128 rows][8]; 0 if none
   // backward dK/dV: per-head key order [B, H, N] i32, item records [n_slots] int4 {qlo, steps, keys,
   // perm offset}, items by length [n_slots] + count i32, f32 partial dK_h, dV_h [2][B, H, N, d]
   size_t off_dkv_perm, off_dkv_slots, off_dkv_items, off_dkv_part;

@@ -147,6 +147,24 @@ DMA_DEVINL void store_row32(uint16_t* dst, const float (&v)[32]) {
     *reinterpret_cast<uint4*>(dst + u) = w;
   }
 }
+// The low-order parts v - bf16(v) of 32 outputs, as bf16: with the row stored by store_row32,
+// hi + lo carries v to about 16 significant bits.  Blocked layout: the 8-column group k of row r of
+// a 128-row block sits at dst_k + r * 8 (dst_k = the group's [128][8] slice), so that the 32 lanes
+// of a warp, 32 consecutive rows, store 512 contiguous bytes per instruction.
+DMA_DEVINL void store_row32_lo(uint16_t* group0, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 32; u += 8) {
+    float q[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) q[k] = v[u + k] - bf16_to_f32(f32_to_bf16(v[u + k]));
+    uint4 w;
+    w.x = pack_bf16x2(q[0], q[1]);
+    w.y = pack_bf16x2(q[2], q[3]);
+    w.z = pack_bf16x2(q[4], q[5]);
+    w.w = pack_bf16x2(q[6], q[7]);
+    *reinterpret_cast<uint4*>(group0 + (size_t)(u / 8) * 128 * 8 + (size_t)r * 8) = w;
+  }
+}
 DMA_DEVINL void store_row32(float* dst, const float (&v)[32]) {
 #pragma unroll
   for (int u = 0; u < 32; u += 4) *reinterpret_cast<float4*>(dst + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);

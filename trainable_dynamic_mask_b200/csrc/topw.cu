@@ -140,9 +140,10 @@ constexpr int kThWarps = kThThreads / 32;
 // over chunks.  One CTA per row.
 __global__ void __launch_bounds__(kThThreads)
 topw_thresh_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in, int32_t* __restrict__ T_out,
-                   int N, int w) {
+                   int N, int w_max, const int32_t* __restrict__ w_heads, int H) {
   extern __shared__ __align__(16) uint32_t table[];   // [nch][nch + 1]
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int w = row_window(w_heads, row, H, w_max);
   const int nch = (N + kC - 1) / kC, cw = nch + 1;
   const int32_t* prow = p_in + (size_t)row * N;
   const int32_t* rrow = rank_in + (size_t)row * N;
@@ -220,7 +221,7 @@ constexpr int kEvThreads = 128;
 __global__ void __launch_bounds__(kEvThreads)
 topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in,
                   const int32_t* __restrict__ T_in, int32_t* __restrict__ evict, int32_t* __restrict__ status,
-                  int N, int w) {
+                  int N, int w_max, const int32_t* __restrict__ w_heads, int H) {
   constexpr int kEvU = 4;            // ranks scanned per thread per round
   __shared__ __align__(16) int32_t crank[kC];   // ranks of the chunk's own keys (INT_MAX past the end)
   __shared__ int32_t L[kC];          // old candidates, ascending rank
@@ -228,6 +229,7 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   __shared__ int32_t wcount[kEvU][kEvThreads / 32];
   const int k = blockIdx.x, row = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int w = row_window(w_heads, row, H, w_max);
   const int nch = (N + kC - 1) / kC;
   const int t0 = k * kC, t1 = min(t0 + kC, N);
   const int32_t* prow = p_in + (size_t)row * N;
@@ -641,14 +643,15 @@ DMA_DEVINL void sel_find_bin(SelShared& S, uint32_t need, int nbins, int tid) {
 // w-th best key has at most kSelCand keys; those are then resolved in shared memory.  A last pass
 // writes the selected positions in ascending order.
 __global__ void __launch_bounds__(kSelThreads, 2)
-topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int N, int w) {
+topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int N, int w_max,
+                   const int32_t* __restrict__ w_heads, int H, int sel_stride) {
   extern __shared__ __align__(16) unsigned char sel_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(sel_raw);
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* drow = delta + (size_t)row * N;
-  const int k = min(w, N);
-  int32_t* out = sel + (size_t)row * k;
+  const int k = min(row_window(w_heads, row, H, w_max), N);
+  int32_t* out = sel + (size_t)row * sel_stride;
   if (k == N) {
     for (int i = tid; i < N; i += kSelThreads) out[i] = i;
     return;
@@ -847,9 +850,10 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
   if (e != cudaSuccess) return e;
   const int tsmem = nch * (nch + 1) * (int)sizeof(uint32_t);
   { cudaError_t ea = ensure_smem_limit(topw_thresh_kernel, tsmem); if (ea != cudaSuccess) return ea; }
-  topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w);
+  topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w, P.w_heads, P.H);
   topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
-                                                            ws_ptr<int32_t>(ws, P.off_status), P.N, P.w);
+                                                            ws_ptr<int32_t>(ws, P.off_status), P.N, P.w,
+                                                            P.w_heads, P.H);
   const int kp0 = P.q0 / kPairQ;
   topw_lists_kernel<<<dim3(P.n_pairs - kp0, rows), kListThreads, 0, s>>>(
       evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
@@ -862,19 +866,22 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
 // ---------------------------------------------------------------- decode: one key appended
 constexpr int kAppThreads = 256;
 
-// One CTA per (b, h) row: the selection over [0, L) from the one over [0, L-1) (stride w when
-// L - 1 > w; every key when L - 1 <= w, then not read).  The worst selected key is the smallest
+// One CTA per (b, h) row: the selection over [0, L) from the one over [0, L-1) (rows of sel_stride
+// entries; the row's window w holds its w keys when L - 1 > w, every key 0 .. L-2 when L - 1 <= w,
+// then not read).  The worst selected key is the smallest
 // (order key, ~index) composite: the smallest delta, the larger index among equal ones.  The new
 // key L - 1 enters iff its order key is strictly larger; it then has the largest index, so the
 // ascending list loses the worst key's entry and gains L - 1 at its end.
 __global__ void __launch_bounds__(kAppThreads)
-topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int L, int w) {
+topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int L, int w_max,
+                   const int32_t* __restrict__ w_heads, int H, int sel_stride) {
   __shared__ uint64_t wmin[kAppThreads / 32];
   __shared__ int pos;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* drow = delta + (size_t)row * L;
-  const int kp = min(L - 1, w), k = min(L, w);
-  int32_t* out = sel + (size_t)row * k;
+  const int w = row_window(w_heads, row, H, w_max);
+  const int kp = min(L - 1, w);
+  int32_t* out = sel + (size_t)row * sel_stride;
   if (kp < w) {   // every key is selected
     for (int i = tid; i < L; i += kAppThreads) out[i] = i;
     return;
@@ -918,14 +925,16 @@ topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
 }
 
 cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
-  topw_append_kernel<<<P.B * P.H, kAppThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w);
+  topw_append_kernel<<<P.B * P.H, kAppThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w,
+                                                       P.w_heads, P.H, P.sel_len);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
   const int smem = (int)sizeof(SelShared);
   { cudaError_t ea = ensure_smem_limit(topw_decode_kernel, smem); if (ea != cudaSuccess) return ea; }
-  topw_decode_kernel<<<P.B * P.H, kSelThreads, smem, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w);
+  topw_decode_kernel<<<P.B * P.H, kSelThreads, smem, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w,
+                                                          P.w_heads, P.H, P.sel_len);
   return cudaGetLastError();
 }
 
