@@ -371,7 +371,7 @@ def run_ours(args, world, rank):
     }
     legs = [] if args.no_legs else [x for x in args.legs.split(",") if x]
     if legs:
-        run = {"decode": leg_decode, "train": leg_train, "chunk": leg_chunk, "long": leg_long}
+        run = {"decode": leg_decode, "train": leg_train, "chunk": leg_chunk, "long": leg_long, "cp": leg_cp}
         line["legs"] = {name: run[name](args, world, torch, dma, peaks) for name in legs}
         line["gpu_launches"] += sum(leg["gpu_launches"] for leg in line["legs"].values())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -640,6 +640,101 @@ def leg_long(args, world, torch, dma, peaks):
     return out
 
 
+def leg_cp(args, world, torch, dma, peaks):
+    """Context-parallel prefill of the long workload over R = 2 shards, the ranks emulated one after
+    another on this GPU: phase A per rank (gate on the shard, its candidates), the exchange (an
+    all-gather of R candidate buffers: not run here, its bytes reported), phase B per rank (prefix
+    stand-in, selection and attention of the shard's queries).  The step of R GPUs would take
+    max_r A_r + exchange + max_r B_r."""
+    import numpy as np
+
+    from trainable_dynamic_mask_b200 import cp
+    from workloads import get, make_inputs
+    R = 2
+    wl = get("long")
+    I = make_inputs(wl)
+    Q, K, V = (_to_dev_bf16(I.bits[n], torch) for n in ("Q", "K", "V"))
+    Dl = _to_dev_bf16(I.bits["Delta"], torch)
+    A = torch.from_numpy(I.A).cuda()
+    del I
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ranks = []
+    for r, (s0, s1) in enumerate(cp.shard_bounds(wl.N, R)):
+        n = s1 - s0
+        p = dma.make_params(wl.B, wl.H, wl.Hkv, n, wl.d, wl.w, dtype="bf16")
+        lay = dma.cp_layout(p, s0, r)
+        Pr = lay.prefix_rows
+        Nc = Pr + n
+        p2 = dma.make_params(wl.B, wl.H, wl.Hkv, Nc, wl.d, wl.w, Nq=n, dtype="bf16", forward_only=True)
+        x = {"p": p, "p2": p2, "s0": s0, "n": n, "lay": lay, "Nc": Nc,
+             "Q": Q[:, :, s0:s1].contiguous(), "K": K[:, :, s0:s1].contiguous(), "V": V[:, :, s0:s1].contiguous(),
+             "delta": torch.empty((wl.B, wl.H, n), dtype=torch.float32, device="cuda"),
+             "cand": torch.empty(lay.cand_bytes, dtype=torch.uint8, device="cuda"),
+             "ws": torch.zeros(lay.ws_bytes, dtype=torch.uint8, device="cuda"),
+             "dc": torch.empty((wl.B, wl.H, Nc), dtype=torch.float32, device="cuda"),
+             "Kc": torch.empty((wl.B, wl.Hkv, Nc, wl.d), dtype=torch.bfloat16, device="cuda"),
+             "Vc": torch.empty((wl.B, wl.Hkv, Nc, wl.d), dtype=torch.bfloat16, device="cuda"),
+             "pc": torch.empty((wl.B, wl.Hkv, Nc), dtype=torch.int32, device="cuda"),
+             "ws2": dma.alloc_workspace(p2),
+             "ev": torch.empty((wl.B, wl.H, Nc), dtype=torch.int32, device="cuda"),
+             "O": torch.empty((wl.B, wl.H, n, wl.d), dtype=torch.bfloat16, device="cuda"),
+             "LSE": torch.empty((wl.B, wl.H, n), dtype=torch.float32, device="cuda")}
+        ranks.append(x)
+    allc = torch.empty((R, ranks[0]["lay"].cand_bytes), dtype=torch.uint8, device="cuda")
+
+    def phase_a(x):
+        dma.gate(x["p"], x["V"], Dl, A, x["delta"], None, None)
+        dma.cp_candidates(x["p"], x["s0"], x["delta"], x["K"], x["V"], x["cand"], x["ws"])
+
+    def phase_b(x, r):
+        dma.cp_compact(x["p"], x["s0"], r, allc[:r] if r else None, x["delta"], x["K"], x["V"], x["dc"], x["Kc"],
+                       x["Vc"], x["pc"], x["ws"])
+        dma.topk_mask(x["p2"], x["dc"], x["ev"], x["ws2"])
+        dma.attn_fwd(x["p2"], x["Q"], x["Kc"], x["Vc"], x["dc"], x["ev"], x["ws2"], x["O"], x["LSE"])
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    n_rep = max(3, min(args.steps // 50, 10))
+    ta = [[] for _ in range(R)]
+    tb = [[] for _ in range(R)]
+    for rep in range(2 + n_rep):
+        for r, x in enumerate(ranks):
+            t = timed(lambda: phase_a(x))
+            allc[r].copy_(x["cand"])          # the exchange's result (an all-gather across GPUs)
+            if rep >= 2:
+                ta[r].append(t)
+        torch.cuda.synchronize()
+        for r, x in enumerate(ranks):
+            t = timed(lambda: phase_b(x, r))
+            if rep >= 2:
+                tb[r].append(t)
+    A_ms = [statistics.median(v) for v in ta]
+    B_ms = [statistics.median(v) for v in tb]
+    step_ms = max(A_ms) + max(B_ms)
+    flops = 4.0 * wl.d * wl.kept_pairs()
+    cb = ranks[0]["lay"].cand_bytes
+    return {"metric": "context-parallel long prefill kept-pair TFLOP/s (R = 2 shards, ranks emulated on one GPU, "
+                      "exchange not included)",
+            "value": round(flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "config": {"workload": "long", "shards": R, "B": wl.B, "H": wl.H, "Hkv": wl.Hkv, "N": wl.N, "d": wl.d,
+                       "w": wl.w, "compacted_keys_per_rank": [x["Nc"] for x in ranks]},
+            "phase_a_us": [round(t * 1e3, 2) for t in A_ms], "phase_b_us": [round(t * 1e3, 2) for t in B_ms],
+            "step_us_without_exchange": round(step_ms * 1e3, 2),
+            "exchange_bytes_received_per_rank": R * cb, "candidate_buffer_bytes": cb,
+            "exchange_us_at_measured_nvlink_770_GBps": round(R * cb / 770e9 * 1e6, 2),
+            "note": "unmeasured on more than one GPU: the runs of this build have one GPU",
+            # per timed repetition: phase A 3 kernels per rank; phase B 7 on rank 0 (copy of its own rows,
+            # top-w 5, attention) and 10 on rank 1 (merged selection: gather, select, union, then the same)
+            "gpu_launches": (3 + 7 + 3 + 10) * n_rep}
+
+
 def leg_train(args, world, torch, dma, peaks):
     """Training step on the train workload: gate (saving x) + mask + attention
     forward + attention backward + gate backward.  kept-pair FLOPs = 14 d pairs
@@ -825,8 +920,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-legs", action="store_true", help="skip the decode and training legs")
-    ap.add_argument("--legs", default="long,decode,train,chunk",
-                    help="comma-separated legs to run: long, decode, train, chunk")
+    ap.add_argument("--legs", default="long,decode,train,chunk,cp",
+                    help="comma-separated legs to run: long, decode, train, chunk, cp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--clock-soak", type=float, default=1.5,

@@ -288,6 +288,66 @@ dma_status_t dma_gate_bwd_noalloc(const dma_params_t* p, const void* V, const vo
                                   void* stream);
 
 /*
+ * Context-parallel prefill: the sequence split into contiguous shards, one per rank (GPU), with one
+ * exchange of each shard's best keys.  Reading of the m_t equation (section "Dynamic Sparse Mask
+ * Generation"): a query keeps the best min(t+1, w) keys of [0, t] by delta, ties to the lower
+ * position; the best keys of a union are among the best keys of its parts, so every query of shard r
+ * selects within (the best keys of the prefix in front of the shard) + (the shard's own keys), and
+ * the best keys of that prefix lie among the best keys of each earlier shard.  The page names no
+ * multi-GPU scheme; this follows from the equation alone.
+ *
+ * Per rank r, with p the shard problem (N = the shard's length len, every other field as for the
+ * whole sequence; w_heads allowed; Nq is ignored):
+ *   1. dma_gate on the shard (delta is per position);
+ *   2. dma_cp_candidates: the shard's candidate buffer (cand_bytes, the same on every rank);
+ *   3. the exchange: every rank receives the candidate buffers of the ranks before it (an all-gather
+ *      of the fixed-size buffers, e.g. NCCL);
+ *   4. dma_cp_compact: from those n_prev buffers, the compacted sequence of P + len rows (P =
+ *      prefix_rows = min(G w, prefix_len), prefix_len = the shard's first position);
+ *   5. dma_topk_mask and dma_attn_fwd on the compacted sequence as a chunk of queries: N = P + len,
+ *      Nq = len, K = Kc, V = Vc, delta = delta_c.  The shard's O and LSE equal the rows of the whole
+ *      sequence's (selection bit for bit; attention within rounding).
+ *
+ * Layout of a candidate buffer (offsets from dma_cp_layout): pos int32 [B, H, w] (global positions,
+ * ascending per row, -1 past the row's min(W_h, len) keys), delta float32 [B, H, w] (-inf past them),
+ * K and V rows [B, H, w, d] in the storage dtype (zero past them; the rows of head h's KV head).
+ * The workspace of both calls is ws_bytes long; its first int32 is a status word (0 = ok) that
+ * dma_cp_compact ORs 0x20000000 into if a group's union exceeds its P rows (an internal consistency
+ * check; the union holds at most min(G w, prefix_len) keys): clear it before the first call.
+ * Limits: the shard problem's (len <= 16384), G w <= 16384, G <= 255, n_prev w < 2^24.
+ */
+typedef struct {
+  size_t cand_bytes;   /* one shard's candidate buffer */
+  size_t off_pos, off_delta, off_k, off_v;
+  size_t ws_bytes;     /* workspace of dma_cp_candidates and dma_cp_compact */
+  size_t off_status;   /* the workspace's status word */
+  int32_t prefix_rows; /* P = min(G w, prefix_len) */
+  int32_t reserved;
+} dma_cp_layout_t;
+
+/* Sizes and offsets for shard problem p with a prefix of prefix_len positions held by n_prev earlier
+ * shards (both 0 for the first shard). */
+dma_status_t dma_cp_layout(const dma_params_t* p, int32_t prefix_len, int32_t n_prev, dma_cp_layout_t* layout);
+
+/* Candidate buffer of a shard starting at global position shard_start: delta [B, H, len] float32,
+ * K, V [B, Hkv, len, d] dtype (the shard's rows). */
+dma_status_t dma_cp_candidates(const dma_params_t* p, int32_t shard_start, const float* delta, const void* K,
+                               const void* V, void* cand, size_t cand_bytes, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Compacted sequence of a shard from the candidate buffers of the n_prev shards before it (back to
+ * back in shard order in `cands`, cand_bytes each), holding prefix_len positions together:
+ *   delta_c [B, H, P + len] float32, Kc, Vc [B, Hkv, P + len, d] dtype, pos_c [B, Hkv, P + len] int32
+ *   (the original position of every row, -1 for padding).  Rows [0, P): P - |U| padding rows (zero
+ *   K, V; delta -inf), then the union U, ascending in position, over the heads of the group of each
+ *   head's best min(W_h, prefix_len) keys of the prefix (delta -inf for a head that did not select the
+ *   key); rows [P, P + len): the shard's own keys. */
+dma_status_t dma_cp_compact(const dma_params_t* p, int32_t prefix_len, int32_t n_prev, const void* cands,
+                            size_t cands_bytes, const float* delta, const void* K, const void* V, float* delta_c,
+                            void* Kc, void* Vc, int32_t* pos_c, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
  * Reads the device status word of `workspace` (synchronises `stream`).  Returns DMA_OK or
  * DMA_ERR_TIMEOUT when a kernel's bounded wait gave up; *code receives the raw word.
  * dma_clear_device_status resets it (asynchronously on `stream`).

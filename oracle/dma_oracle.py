@@ -58,6 +58,10 @@ __all__ = [
     "head_windows",
     "topw_eviction_heads",
     "decode_select_heads",
+    "cp_candidates",
+    "cp_prefix_len",
+    "cp_compact",
+    "cp_shard_bounds",
 ]
 
 
@@ -458,3 +462,108 @@ def decode_select_heads(delta: np.ndarray, w_heads, w: int) -> list:
     B, H, L = delta.shape
     W = head_windows(w_heads, w)
     return [decode_select(delta[b:b + 1, h:h + 1], int(W[h]))[0, 0] for b in range(B) for h in range(H)]
+
+
+# ----------------------------------------------------------------------------
+# Context-parallel prefill: the sequence split into contiguous shards, one per
+# rank, with a single exchange of each shard's best keys
+# ----------------------------------------------------------------------------
+#
+# The m_t equation selects, for a query at position t, the best min(t+1, W)
+# keys of [0, t] by (delta desc, position asc).  The best keys of a union are
+# among the best keys of its parts, so the best keys of the prefix [0, s_r) in
+# front of shard r are among the best min(W, len_q) keys of every earlier shard
+# q: each shard publishes those candidates once, and rank r rebuilds an exact
+# stand-in for the prefix from the candidates of the shards before it.
+
+def cp_candidates(delta, K, V, w_heads, w: int, shard_start: int):
+    """The candidates a shard publishes: for every (b, h), the best
+    min(W_h, len) keys of the shard by (delta desc, position asc), listed in
+    ascending position, with their global position, delta and the K and V rows
+    of head h's key/value head.  Entries past a row's count hold position -1,
+    delta -inf and zero rows.
+
+    delta [B, H, len], K, V [B, Hkv, len, d] (the shard's part).  Returns a dict
+    pos [B, H, w] int64, delta [B, H, w] float32, K, V [B, H, w, d]."""
+    B, H, L = delta.shape
+    Hkv, d = K.shape[1], K.shape[3]
+    G = H // Hkv
+    W = head_windows(np.full(H, w) if w_heads is None else w_heads, w)
+    pos = np.full((B, H, w), -1, dtype=np.int64)
+    dl = np.full((B, H, w), -np.inf, dtype=np.float32)
+    Kc = np.zeros((B, H, w, d), dtype=K.dtype)
+    Vc = np.zeros((B, H, w, d), dtype=V.dtype)
+    for b in range(B):
+        for h in range(H):
+            sel = decode_select(delta[b:b + 1, h:h + 1], int(W[h]))[0, 0]   # ascending shard positions
+            k = sel.size
+            pos[b, h, :k] = shard_start + sel
+            dl[b, h, :k] = np.asarray(delta[b, h, sel], dtype=np.float32)
+            Kc[b, h, :k] = K[b, h // G, sel]
+            Vc[b, h, :k] = V[b, h // G, sel]
+    return {"pos": pos, "delta": dl, "K": Kc, "V": Vc}
+
+
+def cp_prefix_len(G: int, w: int, prefix_len: int) -> int:
+    """Rows that stand in for the prefix of a shard: min(G w, prefix_len)."""
+    return min(G * w, prefix_len)
+
+
+def cp_compact(cands, prefix_len: int, delta, K, V, w_heads, w: int):
+    """The compacted sequence rank r attends over: a stand-in for the prefix
+    [0, prefix_len) followed by the shard's own keys.
+
+    cands: the cp_candidates of every earlier shard, in shard order.  For each
+    (b, h) the best min(W_h, prefix_len) of the merged candidates (delta desc,
+    position asc) are the best keys of the whole prefix.  For each (b, g) the
+    stand-in holds the union of those sets over the heads of group g, ascending
+    in position, after P - |union| padding rows (P = cp_prefix_len): padding
+    rows have zero K and V and delta -inf for every head; a union key that head
+    h did not select has delta -inf for head h.  Then the shard's own keys.
+
+    Returns (K_c, V_c [B, Hkv, P + len, d], delta_c [B, H, P + len], P,
+    pos_c [B, Hkv, P + len]: the original position of every row, -1 for padding)."""
+    B, H, L = delta.shape
+    Hkv, d = K.shape[1], K.shape[3]
+    G = H // Hkv
+    W = head_windows(np.full(H, w) if w_heads is None else w_heads, w)
+    P = cp_prefix_len(G, w, prefix_len)
+    Kc = np.zeros((B, Hkv, P + L, d), dtype=K.dtype)
+    Vc = np.zeros((B, Hkv, P + L, d), dtype=V.dtype)
+    dc = np.full((B, H, P + L), -np.inf, dtype=np.float32)
+    Kc[:, :, P:] = K
+    Vc[:, :, P:] = V
+    dc[:, :, P:] = delta
+    pc = np.full((B, Hkv, P + L), -1, dtype=np.int64)
+    pc[:, :, P:] = prefix_len + np.arange(L)
+    for b in range(B):
+        for g in range(Hkv):
+            chosen = {}     # position -> (K row, V row, {head: delta})
+            for hh in range(G):
+                h = g * G + hh
+                pos = np.concatenate([c["pos"][b, h] for c in cands]) if cands else np.zeros(0, np.int64)
+                dl = np.concatenate([c["delta"][b, h] for c in cands]) if cands else np.zeros(0, np.float32)
+                kr = np.concatenate([c["K"][b, h] for c in cands]) if cands else np.zeros((0, d))
+                vr = np.concatenate([c["V"][b, h] for c in cands]) if cands else np.zeros((0, d))
+                real = np.nonzero(pos >= 0)[0]
+                order = sorted(real, key=lambda i: (-float(dl[i]), int(pos[i])))
+                for i in order[:min(int(W[h]), prefix_len)]:
+                    ent = chosen.setdefault(int(pos[i]), (kr[i], vr[i], {}))
+                    ent[2][h] = dl[i]
+            keys = sorted(chosen)
+            assert len(keys) <= P
+            base = P - len(keys)
+            for n, j in enumerate(keys):
+                kr, vr, dh = chosen[j]
+                Kc[b, g, base + n] = kr
+                Vc[b, g, base + n] = vr
+                pc[b, g, base + n] = j
+                for h, v in dh.items():
+                    dc[b, h, base + n] = v
+    return Kc, Vc, dc, P, pc
+
+
+def cp_shard_bounds(N: int, R: int):
+    """Contiguous shards of [0, N) for R ranks: shard r = [r n, min((r+1) n, N)), n = ceil(N / R)."""
+    n = -(-N // R)
+    return [(min(r * n, N), min((r + 1) * n, N)) for r in range(R)]

@@ -179,6 +179,23 @@ assert lib.dma_selftest_bounded_wait(pp, FAKE, need - 1, 1000, None) == WORKSPAC
 # gate_append(p, V, Delta, A, delta, x_save, stream)
 assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, None, None, None) == INVALID
 assert lib.dma_gate_append(ctypes.byref(pd), FAKE, FAKE, FAKE, FAKE, FAKE + 4, None) == INVALID
+# context-parallel prefill: layout arguments, buffer sizes and workspace checked on the host
+pc2 = dma.make_params(1, 4, 2, 500, 128, 64)
+lay = dma._lib.DmaCpLayout()
+assert lib.dma_cp_layout(ctypes.byref(pc2), 100, 0, ctypes.byref(lay)) == INVALID      # a prefix needs shards
+assert lib.dma_cp_layout(ctypes.byref(pc2), 0, 1, ctypes.byref(lay)) == INVALID
+assert lib.dma_cp_layout(ctypes.byref(pc2), 1000, 2, ctypes.byref(lay)) == OK and lay.prefix_rows == 128
+assert lib.dma_cp_layout(ctypes.byref(pc2), 90, 1, ctypes.byref(lay)) == OK and lay.prefix_rows == 90
+big = dma.make_params(1, 8, 1, 500, 128, 4096)                                      # G w = 32768 > 16384
+assert lib.dma_cp_layout(ctypes.byref(big), 0, 0, ctypes.byref(lay)) == UNSUPPORTED
+assert lib.dma_cp_layout(ctypes.byref(pc2), 0, 0, ctypes.byref(lay)) == OK
+cb, wb = lay.cand_bytes, lay.ws_bytes
+assert cb == 1024 + 1024 + 2 * (4 * 64 * 128 * 2)   # pos, delta, K rows, V rows of B H w = 4 x 64 entries
+assert lib.dma_cp_candidates(ctypes.byref(pc2), 0, FAKE, FAKE, FAKE, FAKE, cb - 1, FAKE, wb, None) == INVALID
+assert lib.dma_cp_candidates(ctypes.byref(pc2), 0, FAKE, FAKE, FAKE, FAKE, cb, FAKE, wb - 1, None) == WORKSPACE
+assert lib.dma_cp_candidates(ctypes.byref(pc2), -1, FAKE, FAKE, FAKE, FAKE, cb, FAKE, wb, None) == INVALID
+assert lib.dma_cp_compact(ctypes.byref(pc2), 1000, 2, FAKE, 2 * cb - 1, *([FAKE] * 7), FAKE, 1 << 30, None) == INVALID
+assert lib.dma_cp_compact(ctypes.byref(pc2), 1000, 2, None, 2 * cb, *([FAKE] * 7), FAKE, 1 << 30, None) == INVALID
 pdec = dma.make_params(8, 32, 8, 65536, 128, 2048, Nq=1)   # 64 MiB of gx alone: more than the fixed array
 assert lib.dma_gate_bwd_noalloc(ctypes.byref(pdec), *([FAKE] * 9), None) == UNSUPPORTED
 # the gate kernels hold at most 64 query heads; more is refused on the host, not at launch

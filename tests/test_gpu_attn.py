@@ -101,8 +101,9 @@ def test_attn_fwd_full(case):
 
 def test_attn_fwd_forward_only_flag_same_outputs():
     """DMA_FLAG_FORWARD_ONLY changes what the forward keeps for a backward, never its outputs:
-    O and LSE bit for bit equal to those of the same problem without the flag."""
-    wl = get("prefill").with_(H=4, Hkv=2, N=1500, seed=27)
+    O and LSE bit for bit equal to those of the same problem without the flag (a shape whose pairs
+    are not split, so that no merge order can differ between the two runs)."""
+    wl = get("prefill").with_(H=32, Hkv=8, seed=27)
     dma, torch, I, p, ws, dev, d32, e_ref = _setup(wl)
     O, LSE = _fwd(dma, torch, wl, p, ws, dev)
     p1 = dma.make_params(wl.B, wl.H, wl.Hkv, wl.N, wl.d, wl.w, dtype=wl.dtype, forward_only=True)
@@ -110,8 +111,9 @@ def test_attn_fwd_forward_only_flag_same_outputs():
     dma.topk_mask(p1, dev["delta"], dev["evict"], ws1)
     O1, LSE1 = _fwd(dma, torch, wl, p1, ws1, dev)
     assert torch.equal(O.view(torch.int16), O1.view(torch.int16)) and torch.equal(LSE, LSE1)
-    O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, gemm_dtype=np.float32)
-    assert_close(to_np(O1), O_ref, "O")
+    rows = _sample_rows(wl.N, 512, 98)
+    O_ref, L_ref = oracle.attn_fwd(I.Q, I.K, I.V, d32.astype(np.float64), e_ref, rows=rows, gemm_dtype=np.float32)
+    assert_close(to_np(O1)[:, :, rows], O_ref[:, :, rows], "O")
 
 
 def _sample_rows(N, n, seed):

@@ -133,3 +133,24 @@ def test_append_tie_mistakes_are_caught(monkeypatch, ge, smaller):
     monkeypatch.setattr(oracle, "decode_select_append", _append_with(ge, smaller))
     assert _fails(TA.test_decode_select_append_equals_the_full_selection_at_every_length) or \
         _fails(TA.test_decode_select_append_cases)
+
+
+def test_candidates_of_the_previous_shard_only_are_caught(monkeypatch):
+    """A sharded prefill that merges only the shard just before instead of every earlier one."""
+    import test_oracle_cp as TC
+    real = od.cp_compact
+
+    def bad(cands, prefix_len, *a, **k):
+        return real(cands[-1:], prefix_len, *a, **k)
+
+    monkeypatch.setattr(oracle, "cp_compact", bad)
+    assert _fails(TC.test_sharded_equals_whole_sequence, 3, 37, None)
+
+
+def test_prefix_stand_in_of_one_window_is_caught(monkeypatch):
+    """A stand-in of w rows for the prefix (one head's window) instead of G w: the union of the
+    group's heads does not fit."""
+    import test_oracle_cp as TC
+    monkeypatch.setattr(oracle, "cp_prefix_len", lambda G, w, prefix_len: min(w, prefix_len))
+    monkeypatch.setattr(od, "cp_prefix_len", lambda G, w, prefix_len: min(w, prefix_len))
+    assert _fails(TC.test_sharded_equals_whole_sequence, 2, 37, None)

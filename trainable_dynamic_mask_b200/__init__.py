@@ -13,8 +13,8 @@ from __future__ import annotations
 
 import ctypes
 
-from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DMA_FLAG_FORWARD_ONLY, DmaError, DmaParams, DmaWsLayout, LIB_PATH, check,
-                   exported_names, load)
+from ._lib import (BLOCK_Q, DMA_BF16, DMA_F32, DMA_FLAG_FORWARD_ONLY, DmaCpLayout, DmaError, DmaParams, DmaWsLayout,
+                   LIB_PATH, check, exported_names, load)
 
 __all__ = [
     "BLOCK_Q", "DMA_BF16", "DMA_F32", "DmaError", "DmaParams", "LIB_PATH", "load", "exported_names",
@@ -22,7 +22,7 @@ __all__ = [
     "attn_fwd", "attn_bwd",
     "gate_bwd", "gate_bwd_noalloc", "check_device_status", "clear_device_status", "selftest_bounded_wait",
     "abi_version", "alloc_workspace", "forward",
-    "backward",
+    "backward", "cp_layout", "cp_candidates", "cp_compact",
 ]
 
 
@@ -150,6 +150,28 @@ def selftest_bounded_wait(p, workspace, limit_cycles=1_000_000, stream=None):
 def clear_device_status(p, workspace, stream=None):
     check("dma_clear_device_status", load().dma_clear_device_status(ctypes.byref(p), _ptr(workspace),
                                                                     _stream(stream)))
+
+
+# ---------------------------------------------------------------- context-parallel prefill
+
+def cp_layout(p, prefix_len, n_prev) -> DmaCpLayout:
+    """Candidate-buffer and workspace sizes of shard problem p (see trainable_dynamic_mask_b200.cp)."""
+    lay = DmaCpLayout()
+    check("dma_cp_layout", load().dma_cp_layout(ctypes.byref(p), int(prefix_len), int(n_prev), ctypes.byref(lay)))
+    return lay
+
+
+def cp_candidates(p, shard_start, delta, K, V, cand, workspace, stream=None):
+    check("dma_cp_candidates", load().dma_cp_candidates(ctypes.byref(p), int(shard_start), _ptr(delta), _ptr(K),
+                                                        _ptr(V), _ptr(cand), _nbytes(cand), _ptr(workspace),
+                                                        _nbytes(workspace), _stream(stream)))
+
+
+def cp_compact(p, prefix_len, n_prev, cands, delta, K, V, delta_c, Kc, Vc, pos_c, workspace, stream=None):
+    check("dma_cp_compact", load().dma_cp_compact(ctypes.byref(p), int(prefix_len), int(n_prev), _ptr(cands),
+                                                  _nbytes(cands), _ptr(delta), _ptr(K), _ptr(V), _ptr(delta_c),
+                                                  _ptr(Kc), _ptr(Vc), _ptr(pos_c), _ptr(workspace),
+                                                  _nbytes(workspace), _stream(stream)))
 
 
 # ---------------------------------------------------------------- convenience (torch allocation)

@@ -38,6 +38,11 @@ class DmaWsLayout(ctypes.Structure):
                 ("reserved", c_i32)]
 
 
+class DmaCpLayout(ctypes.Structure):
+    _fields_ = [("cand_bytes", c_sz), ("off_pos", c_sz), ("off_delta", c_sz), ("off_k", c_sz), ("off_v", c_sz),
+                ("ws_bytes", c_sz), ("off_status", c_sz), ("prefix_rows", c_i32), ("reserved", c_i32)]
+
+
 # name -> argtypes (every function returns dma_status_t as int32 unless listed in _RESTYPES)
 _SIGS = {
     "dma_status_string": [c_i32],
@@ -59,6 +64,10 @@ _SIGS = {
     "dma_check_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp, ctypes.POINTER(c_i32)],
     "dma_clear_device_status": [ctypes.POINTER(DmaParams), c_vp, c_vp],
     "dma_selftest_bounded_wait": [ctypes.POINTER(DmaParams), c_vp, c_sz, ctypes.c_int64, c_vp],
+    "dma_cp_layout": [ctypes.POINTER(DmaParams), c_i32, c_i32, ctypes.POINTER(DmaCpLayout)],
+    "dma_cp_candidates": [ctypes.POINTER(DmaParams), c_i32, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp, c_sz, c_vp],
+    "dma_cp_compact": [ctypes.POINTER(DmaParams), c_i32, c_i32, c_vp, c_sz, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                       c_vp, c_sz, c_vp],
 }
 _RESTYPES = {"dma_status_string": ctypes.c_char_p, "dma_abi_version": c_i32}
 

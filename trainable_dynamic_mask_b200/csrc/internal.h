@@ -101,6 +101,10 @@ cudaError_t launch_gate_fwd(const Plan& P, const void* V, const void* Delta, con
 cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evict, void* ws,
                                 cudaStream_t s);
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s);
+// Top-min(window, N) of each of `rows` rows of N values (delta desc, index asc), ascending indices into
+// sel[row * sel_stride ..]; the row's window is w_heads[row % H] clamped to [1, w] (w when w_heads is null).
+cudaError_t launch_topw_select_rows(const float* delta, int rows, int N, int w, const int32_t* w_heads, int H,
+                                    int32_t* sel, int sel_stride, cudaStream_t s);
 cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s);
 cudaError_t launch_selftest_wait(const Plan& P, void* ws, long long limit_cycles, cudaStream_t s);
 cudaError_t launch_gate_append(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,

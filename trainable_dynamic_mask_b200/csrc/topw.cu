@@ -930,12 +930,17 @@ cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cuda
   return cudaGetLastError();
 }
 
-cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
+cudaError_t launch_topw_select_rows(const float* delta, int rows, int N, int w, const int32_t* w_heads, int H,
+                                    int32_t* sel, int sel_stride, cudaStream_t s) {
   const int smem = (int)sizeof(SelShared);
   { cudaError_t ea = ensure_smem_limit(topw_decode_kernel, smem); if (ea != cudaSuccess) return ea; }
-  topw_decode_kernel<<<P.B * P.H, kSelThreads, smem, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w,
-                                                          P.w_heads, P.H, P.sel_len);
+  topw_decode_kernel<<<rows, kSelThreads, smem, s>>>(delta, sel, N, w, w_heads, H, sel_stride);
   return cudaGetLastError();
+}
+
+cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
+  return launch_topw_select_rows(delta, P.B * P.H, P.N, P.w, P.w_heads, P.H, ws_ptr<int32_t>(ws, P.off_sel),
+                                 P.sel_len, s);
 }
 
 }  // namespace dma
