@@ -396,18 +396,255 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
 
 // Live keys of a range of query rows [t0, t1): j < t1 and e_j > max(j, t0).  The "full" ones
 // (j <= t0 and e_j >= t1: selected by every row of the range) come first, then the others, each
-// group in ascending key order.  One CTA scans the keys of a pair of blocks (kPairQ rows) once and
-// builds three lists from them: those of its two blocks (the mask encoding of the interface) and
-// that of the pair (the attention forward's work item), whose entries also carry e_j - j (the
-// number of queries selecting the key) and delta_j * log2(e), and which is padded to a multiple of
-// 128 entries with key -1 and e - j = 0 (masked for every row).
+// group in ascending key order.  One CTA per (row, pair of blocks) builds three lists: those of its
+// two blocks (the mask encoding of the interface) and that of the pair (the attention forward's work
+// item), whose entries also carry e_j - j (the number of queries selecting the key) and
+// delta_j * log2(e), and which is padded to a multiple of 128 entries with key -1 and e - j = 0
+// (masked for every row).
+//
+// The keys before the pair's first row t0 that are still live at t0 are among the w best keys of
+// [0, t0): the ranks 0 .. T_k of the row (T_k, the rank of the w-th best key of [0, t0), from the
+// thresholds kernel; k = t0 / 128).  So the CTA scans whichever is shorter, those ranks (through the
+// rank -> position map) or the positions [0, t0) -- about w N / t0 against t0 entries -- and then the
+// pair's own positions [t0, t1).  Each list is kept as two bitmaps over positions (full, partial),
+// compacted at the end in ascending order.
 constexpr int kListThreads = 256;
+constexpr int kListWords = kTopwMaxN / 32;   // bitmap words of a whole row
+constexpr int kListStreamMaxN = 4096;        // rows up to this length take the streaming kernel below
+
+__global__ void __launch_bounds__(kListThreads)
+topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
+                  const int32_t* __restrict__ p_in, const int32_t* __restrict__ T_in,
+                  int32_t* __restrict__ counts, int32_t* __restrict__ lists,
+                  int32_t* __restrict__ pcounts, int32_t* __restrict__ plists,
+                  int32_t* __restrict__ plen, float* __restrict__ pdl, int32_t* __restrict__ fcnt, int N,
+                  int list_cap, int pair_cap, int n_blocks, int n_pairs, int kp0) {
+  __shared__ uint32_t bm[6][kListWords];   // list L: bm[2L] full keys, bm[2L + 1] partial keys
+  __shared__ uint32_t wsum3[3][kListThreads / 32];
+  const int kp = kp0 + (int)blockIdx.x, row = blockIdx.y;   // pairs from kp0: the ones holding a query
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = kp * kPairQ;
+  const bool has_b = t0 + kC < N;
+  // list 0: block 2kp, list 1: block 2kp + 1, list 2: the pair
+  const int lo[3] = {t0, t0 + kC, t0};
+  const int hi[3] = {min(t0 + kC, N), min(t0 + kPairQ, N), min(t0 + kPairQ, N)};
+  const int cap[3] = {list_cap, list_cap, pair_cap};
+  const int t1 = hi[2];
+  const int nw = (t1 + 31) / 32;
+  const int32_t* erow = evict + (size_t)row * N;
+  const float* drow = delta + (size_t)row * N;
+  const int32_t* prow = p_in + (size_t)row * N;
+  // the attention forward's merge counters of this pair start at zero for every new mask
+  if (tid < 4) fcnt[((size_t)row * n_pairs + kp) * 4 + tid] = 0;
+  // and its dynamic schedule's counters (after the merge counters of every pair)
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid < 2) fcnt[(size_t)gridDim.y * n_pairs * 4 + tid] = 0;
+  // bit 2L (full) or 2L + 1 (partial) of key j < t1 evicted at e, for each list it is live in
+  auto classify = [&](int j, int e) -> uint32_t {
+    uint32_t m = 0;
+#pragma unroll
+    for (int L = 0; L < 3; ++L) {
+      const bool live = (L != 1 || has_b) && j < hi[L] && e > max(j, lo[L]);
+      const bool full = live && j <= lo[L] && e >= hi[L];
+      if (live) m |= 1u << (2 * L + (full ? 0 : 1));
+    }
+    return m;
+  };
+  for (int i = tid; i < 6 * kListWords; i += kListThreads)
+    if ((i % kListWords) < nw) bm[i / kListWords][i % kListWords] = 0;
+  __syncthreads();
+  const int Tk = T_in[(size_t)row * (n_blocks + 1) + 2 * kp];
+  constexpr int kBatch = 8;   // keys per thread whose loads are issued together
+  if (Tk < N && Tk + 1 < t0) {
+    // the ranks 0 .. T_k: their positions before t0 (bits set one key at a time)
+    for (int r0 = 0; r0 <= Tk; r0 += kListThreads * kBatch) {
+      int jb[kBatch], eb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int r = r0 + u * kListThreads + tid;
+        jb[u] = r <= Tk ? prow[r] : INT_MAX;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) eb[u] = jb[u] < t0 ? erow[jb[u]] : 0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = jb[u];
+        if (j < t0) {
+          const uint32_t m = classify(j, eb[u]);
+#pragma unroll
+          for (int b = 0; b < 6; ++b)
+            if ((m >> b) & 1u) atomicOr(&bm[b][j >> 5], 1u << (j & 31));
+        }
+      }
+    }
+  } else {
+    // the positions [0, t0) (t0 is a multiple of 256: every warp's 32 positions are a whole word)
+    for (int base0 = 0; base0 < t0; base0 += kListThreads * kBatch) {
+      int eb[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = base0 + u * kListThreads + warp * 32 + lane;
+        eb[u] = j < t0 ? erow[j] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int base = base0 + u * kListThreads + warp * 32;
+        if (base >= t0) break;   // warp-uniform
+        const uint32_t m = classify(base + lane, eb[u]);
+#pragma unroll
+        for (int b = 0; b < 6; ++b) {
+          const uint32_t word = __ballot_sync(0xffffffffu, (m >> b) & 1u);
+          if (lane == 0) bm[b][base >> 5] = word;
+        }
+      }
+    }
+  }
+  {
+    // the pair's own positions [t0, t1): one per thread, whole words per warp
+    const int j = t0 + tid;
+    const uint32_t m = j < t1 ? classify(j, erow[j]) : 0u;
+#pragma unroll
+    for (int b = 0; b < 6; ++b) {
+      const uint32_t word = __ballot_sync(0xffffffffu, (m >> b) & 1u);
+      if (lane == 0 && t0 + warp * 32 < t1) bm[b][(t0 >> 5) + warp] = word;
+    }
+  }
+  __syncthreads();
+  // compaction: the bitmaps' bytes are dealt in equal runs of upt consecutive bytes per thread (so
+  // that every thread has about the same number of keys to write, however short the range).  One
+  // block scan of the six counts (packed two per 32-bit word, 16 bits each: a list holds < 2^16 keys)
+  // gives every key its index: full keys of a list first, then its partial keys.
+  const int nbytes = 4 * nw;
+  const int upt = (nbytes + kListThreads - 1) / kListThreads;   // <= 8
+  const int u0 = tid * upt;
+  auto byte_of = [&](int b, int u) -> uint32_t {
+    return u < nbytes ? (bm[b][u >> 2] >> (8 * (u & 3))) & 0xffu : 0u;
+  };
+  uint32_t pk[3] = {0u, 0u, 0u};
+#pragma unroll
+  for (int b = 0; b < 6; ++b) {
+    int c = 0;
+    for (int u = 0; u < upt; ++u) c += __popc(byte_of(b, u0 + u));
+    pk[b >> 1] += (uint32_t)c << (16 * (b & 1));
+  }
+  uint32_t inc[3] = {pk[0], pk[1], pk[2]};
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+    for (int q = 0; q < 3; ++q) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc[q], o);
+      if (lane >= o) inc[q] += y;
+    }
+  }
+  if (lane == 31) {
+#pragma unroll
+    for (int q = 0; q < 3; ++q) wsum3[q][warp] = inc[q];
+  }
+  __syncthreads();
+  int start[6], total[6];
+#pragma unroll
+  for (int b = 0; b < 6; ++b) {
+    const int q = b >> 1, sh = 16 * (b & 1);
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int v = 0; v < kListThreads / 32; ++v) {
+      const int x = (int)((wsum3[q][v] >> sh) & 0xffffu);
+      before += v < warp ? x : 0;
+      tot += x;
+    }
+    start[b] = before + (int)(((inc[q] - pk[q]) >> sh) & 0xffffu);
+    total[b] = tot;
+  }
+  int n_out[3][2];
+#pragma unroll
+  for (int L = 0; L < 3; ++L) {
+    n_out[L][0] = min(total[2 * L], cap[L]);
+    n_out[L][1] = min(total[2 * L + 1], cap[L] - n_out[L][0]);
+  }
+#pragma unroll
+  for (int L = 0; L < 3; ++L) {
+    if (L == 1 && !has_b) continue;
+    int32_t* dst = L == 0 ? lists + ((size_t)row * n_blocks + 2 * kp) * list_cap
+                 : L == 1 ? lists + ((size_t)row * n_blocks + 2 * kp + 1) * list_cap
+                          : plists + ((size_t)row * n_pairs + kp) * pair_cap;
+#pragma unroll
+    for (int kind = 0; kind < 2; ++kind) {
+      const int b = 2 * L + kind;
+      int o = start[b] + (kind == 1 ? n_out[L][0] : 0);
+      const int lim = kind == 0 ? n_out[L][0] : n_out[L][0] + n_out[L][1];
+      for (int u = 0; u < upt; ++u) {
+        uint32_t x = byte_of(b, u0 + u);
+        while (x) {
+          const int jj = 8 * (u0 + u) + __ffs(x) - 1;
+          x &= x - 1;
+          if (o < lim) dst[o] = jj;
+          ++o;
+        }
+      }
+    }
+  }
+  __syncthreads();   // the pair list is complete for the pass below
+  {
+    // the pair list's e_j - j and delta_j log2(e), entry by entry (global writes of this CTA made
+    // before the barrier above are visible to it)
+    const size_t pb = ((size_t)row * n_pairs + kp) * pair_cap;
+    const int n2 = n_out[2][0] + n_out[2][1];
+    for (int i0 = 0; i0 < n2; i0 += kListThreads * kBatch) {
+      int jb[kBatch], eb[kBatch];
+      float db[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kListThreads + tid;
+        jb[u] = i < n2 ? plists[pb + i] : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        eb[u] = jb[u] >= 0 ? erow[jb[u]] : 0;
+        db[u] = jb[u] >= 0 ? drow[jb[u]] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kListThreads + tid;
+        if (i < n2) {
+          plen[pb + i] = eb[u] - jb[u];
+          pdl[pb + i] = db[u] * kLog2e;
+        }
+      }
+    }
+  }
+  const int nlive = n_out[2][0] + n_out[2][1];
+  const int nround = min(pair_cap, (nlive + kC - 1) / kC * kC);
+  {
+    const size_t pb = ((size_t)row * n_pairs + kp) * pair_cap;
+    for (int i = nlive + tid; i < nround; i += kListThreads) {
+      plists[pb + i] = -1;
+      plen[pb + i] = 0;
+      pdl[pb + i] = 0.f;
+    }
+  }
+  if (tid == 0) {
+    int32_t* ca = counts + ((size_t)row * n_blocks + 2 * kp) * 2;
+    ca[0] = n_out[0][0];
+    ca[1] = n_out[0][0] + n_out[0][1];
+    if (has_b) {
+      ca[2] = n_out[1][0];
+      ca[3] = n_out[1][0] + n_out[1][1];
+    }
+    int32_t* cp = pcounts + ((size_t)row * n_pairs + kp) * 2;
+    cp[0] = n_out[2][0];
+    cp[1] = nlive;
+  }
+}
+
+// The same lists by one streaming pass over all keys j < t1 in ascending order (four keys per
+// thread per round, e_j and delta_j loaded a round ahead, packed per-warp counters): no bitmaps and
+// no rank map, cheaper than the kernel above while t1 is short (rows of up to 4096 keys), dearer on
+// long rows, where the ranks up to T_k are far fewer than the positions before t0.
 constexpr int kListWarps = kListThreads / 32;
 constexpr int kListBits = 10;                    // packed per-warp counters (a warp counts <= 128)
 constexpr int kListMask = (1 << kListBits) - 1;
 
 __global__ void __launch_bounds__(kListThreads)
-topw_lists_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
+topw_lists_stream_kernel(const int32_t* __restrict__ evict, const float* __restrict__ delta,
                   int32_t* __restrict__ counts, int32_t* __restrict__ lists,
                   int32_t* __restrict__ pcounts, int32_t* __restrict__ plists,
                   int32_t* __restrict__ plen, float* __restrict__ pdl, int32_t* __restrict__ fcnt, int N,
@@ -855,11 +1092,18 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w,
                                                             P.w_heads, P.H);
   const int kp0 = P.q0 / kPairQ;
-  topw_lists_kernel<<<dim3(P.n_pairs - kp0, rows), kListThreads, 0, s>>>(
-      evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
-      ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
-      ws_ptr<float>(ws, P.off_pdl), ws_ptr<int32_t>(ws, P.off_fcnt), P.N, P.list_cap, P.pair_cap, P.n_blocks,
-      P.n_pairs, kp0);
+  if (P.N > kListStreamMaxN)
+    topw_lists_kernel<<<dim3(P.n_pairs - kp0, rows), kListThreads, 0, s>>>(
+        evict, delta, pbuf, Tbuf, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
+        ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
+        ws_ptr<float>(ws, P.off_pdl), ws_ptr<int32_t>(ws, P.off_fcnt), P.N, P.list_cap, P.pair_cap, P.n_blocks,
+        P.n_pairs, kp0);
+  else
+    topw_lists_stream_kernel<<<dim3(P.n_pairs - kp0, rows), kListThreads, 0, s>>>(
+        evict, delta, ws_ptr<int32_t>(ws, P.off_counts), ws_ptr<int32_t>(ws, P.off_lists),
+        ws_ptr<int32_t>(ws, P.off_pcounts), ws_ptr<int32_t>(ws, P.off_plists), ws_ptr<int32_t>(ws, P.off_plen),
+        ws_ptr<float>(ws, P.off_pdl), ws_ptr<int32_t>(ws, P.off_fcnt), P.N, P.list_cap, P.pair_cap, P.n_blocks,
+        P.n_pairs, kp0);
   return cudaGetLastError();
 }
 
