@@ -494,7 +494,8 @@ def leg_decode(args, world, torch, dma, peaks):
             "select_append_us": round(t_app * 1e3, 2), "append_equals_full_selection": append_ok,
             "roofline": {"kernel": "decode_split+combine", "bound": "hbm", "achieved": round(gbs, 2),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "peak_kind": peaks["source"], "traffic": None,
+                         "peak_kind": peaks["source"], "traffic": _traffic("decode_split", "attn_fwd.cu"),
+                         "traffic_kernel": "decode_split_kernel (the combine reads 1 MB more)",
                          "algorithmic_bytes": bytes_unique, "bytes_if_per_head": bytes_per_head},
             "dense_causal": dense,
             "gpu_launches": 4 * n}
