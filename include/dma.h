@@ -223,8 +223,9 @@ dma_status_t dma_gate_append(const dma_params_t* p, const void* V, const void* D
  *   Q      [B, H, Nq, d] dtype;  K, V [B, Hkv, N, d] dtype;  delta [B, H, N] float32
  *   evict  [B, H, N] int32 from dma_topk_mask (NULL for decode); the workspace must hold the
  *          lists (or selection) dma_topk_mask wrote for the same delta.  Prefill takes delta_j
- *          and e_j from the per-entry copies dma_topk_mask stored with the lists, so a delta
- *          changed after dma_topk_mask is not seen there: run dma_topk_mask again.
+ *          and e_j from the per-entry copies dma_topk_mask stored with the lists, and decode takes
+ *          delta_j from the copy dma_topk_mask / dma_topk_append stored beside the selection, so a
+ *          delta changed after the selection is not seen there: run the selection again.
  *   O      [B, H, Nq, d] dtype out;  LSE [B, H, Nq] float32 out
  * With bfloat16 storage and Nq == N (a problem the backward can take) the call also keeps, in the
  * workspace, the low-order part of every output, O - bf16(O), rounded to bfloat16, which

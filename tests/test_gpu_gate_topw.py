@@ -160,6 +160,17 @@ def test_decode_select_append(L0, L, w, kind):
         torch.cuda.synchronize()
         if n == L or n - L0 < 40 or n % 17 == 0:
             np.testing.assert_array_equal(_sel_of(dma, p, ws), oracle.decode_select(d[:, :, :n], w), err_msg=f"L={n}")
+    # the decode attention reads delta from the copy the appends kept beside the selection
+    rng = np.random.default_rng(L + w)
+    bf = lambda a: torch.from_numpy(a).to("cuda").bfloat16()
+    q, Kc, Vc = (bf(rng.standard_normal(s).astype(np.float32)) for s in ((B, H, 1, 128), (B, H, L, 128), (B, H, L, 128)))
+    O = torch.empty((B, H, 1, 128), dtype=torch.bfloat16, device="cuda")
+    LSE = torch.empty((B, H, 1), dtype=torch.float32, device="cuda")
+    dma.attn_fwd(p, q, Kc, Vc, f32_dev(d), None, ws, O, LSE)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.decode_attn(to_np(q), to_np(Kc), to_np(Vc), d.astype(np.float64), oracle.decode_select(d, w))
+    np.testing.assert_allclose(to_np(LSE)[:, :, 0], l_ref, atol=2e-2, rtol=1e-2)
+    np.testing.assert_allclose(to_np(O)[:, :, 0], o_ref, atol=2e-2, rtol=1e-2)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])

@@ -210,6 +210,7 @@ dma_status_t make_plan(const dma_params_t* p, Plan* P) {
     }
   } else {
     R.off_sel = take(BH * R.sel_len * sizeof(int32_t));
+    R.off_seld = take(BH * R.sel_len * sizeof(float));
     R.off_dec_part = take(BH * R.n_split * (size_t)(R.d + 2) * sizeof(float));
   }
   if (!R.bf16) {

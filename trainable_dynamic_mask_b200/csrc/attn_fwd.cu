@@ -31,7 +31,7 @@ constexpr int kDecThreads = 256;
 template <int D>
 __global__ void __launch_bounds__(kDecThreads)
 decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__ K,
-                    const uint16_t* __restrict__ V, const float* __restrict__ delta,
+                    const uint16_t* __restrict__ V, const float* __restrict__ seld,
                     const int32_t* __restrict__ sel, float* __restrict__ part, int H, int G, int N,
                     int sel_len, int n_split, float scale_log2, int w, const int32_t* __restrict__ w_heads) {
   constexpr int CH = D / 8;                 // 16-byte chunks per row
@@ -46,6 +46,8 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
   const int s = blockIdx.x, bh = blockIdx.y;
   const int b = bh / H, h = bh % H, g = h / G, Hkv = H / G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the combine kernel may be scheduled now: it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const uint16_t* Kg = K + (size_t)(b * Hkv + g) * N * D;
   const uint16_t* Vg = V + (size_t)(b * Hkv + g) * N * D;
   const int k0 = s * kDecodeSplit;
@@ -53,9 +55,10 @@ decode_split_kernel(const uint16_t* __restrict__ Q, const uint16_t* __restrict__
   // row may hold fewer, and splits past its end reduce nothing: m = -inf, l = 0)
   const int n_row = min(row_window(w_heads, bh, H, w), N);
   const int nk = min(kDecodeSplit, n_row - k0);
+  // the split's keys and their delta, stored beside each other by the selection (no gather of delta)
   const int j = tid < nk ? sel[(size_t)bh * sel_len + k0 + tid] : -1;
   idx[tid] = j;
-  const float dl = j >= 0 ? delta[(size_t)bh * N + j] * kLog2e : 0.f;
+  const float dl = j >= 0 ? seld[(size_t)bh * sel_len + k0 + tid] * kLog2e : 0.f;
   for (int c = tid; c < D; c += kDecThreads) qs[c] = bf16_to_f32(Q[(size_t)bh * D + c]);
   __syncthreads();
   // rows of the split: thread sweep over (row, chunk), consecutive threads along a row
@@ -161,6 +164,9 @@ __global__ void decode_combine_kernel(const float* __restrict__ part, OutT* __re
   float* sm_m = cmb;
   float* sm_w = cmb + n_split;
   const int bh = blockIdx.x, tid = threadIdx.x;
+  // launched as a programmatic dependent of the split kernel: wait for its completion (a no-op when
+  // launched in plain stream order)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* pr = part + (size_t)bh * n_split * (D + 2);
   for (int q = tid; q < n_split; q += blockDim.x) {
     sm_m[q] = pr[(size_t)q * (D + 2)];
@@ -198,11 +204,22 @@ cudaError_t launch_dec_t(const Plan& P, const uint16_t* Q, const uint16_t* K, co
     if (ea != cudaSuccess) return ea;
   }
   decode_split_kernel<D><<<dim3(P.n_split, P.B * P.H), kDecThreads, decode_smem_bytes<D>(), s>>>(
-      Q, K, V, delta, ws_ptr<int32_t>(ws, P.off_sel), part, P.H, P.G, P.N, P.sel_len, P.n_split,
+      Q, K, V, ws_ptr<float>(ws, P.off_seld), ws_ptr<int32_t>(ws, P.off_sel), part, P.H, P.G, P.N, P.sel_len, P.n_split,
       P.scale * kLog2e, P.w, P.w_heads);
-  decode_combine_kernel<D, OutT><<<P.B * P.H, D, 2 * P.n_split * sizeof(float), s>>>(part, (OutT*)O, LSE,
-                                                                                      P.n_split);
-  return cudaGetLastError();
+  if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+  // the combine as a programmatic dependent launch: its CTAs are scheduled while the split kernel
+  // finishes and wait on its completion inside (griddepcontrol.wait), hiding the launch gap
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.B * P.H);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 2 * P.n_split * sizeof(float);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D, OutT>, (const float*)part, (OutT*)O, LSE, P.n_split);
 }
 
 }  // namespace

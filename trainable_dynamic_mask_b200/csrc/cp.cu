@@ -342,7 +342,7 @@ dma_status_t dma_cp_candidates(const dma_params_t* p, int32_t shard_start, const
   if (!ok_ptr(workspace) || workspace_bytes < L.ws_bytes) return DMA_ERR_WORKSPACE;
   cudaStream_t s = (cudaStream_t)stream;
   int32_t* sel = ws_ptr<int32_t>(workspace, L.off_sel);
-  cudaError_t e = launch_topw_select_rows(delta, P.B * P.H, P.N, P.w, P.w_heads, P.H, sel, P.w, s);
+  cudaError_t e = launch_topw_select_rows(delta, P.B * P.H, P.N, P.w, P.w_heads, P.H, sel, nullptr, P.w, s);
   if (e != cudaSuccess) return DMA_ERR_CUDA;
   unsigned char* c = static_cast<unsigned char*>(cand);
   cp_pack_kernel<<<dim3(P.B * P.H, (P.w + kCpThreads - 1) / kCpThreads), kCpThreads, 0, s>>>(sel, delta, (const unsigned char*)K, (const unsigned char*)V,
@@ -375,7 +375,7 @@ dma_status_t dma_cp_compact(const dma_params_t* p, int32_t prefix_len, int32_t n
     const size_t n = (size_t)P.B * P.H * n_prev * P.w;
     cp_gather_delta_kernel<<<(unsigned)((n + 255) / 256 < 148 * 8 ? (n + 255) / 256 : 148 * 8), 256, 0, s>>>(
         cb, L.cand_bytes, L.off_delta, dm, P.B * P.H, n_prev, P.w);
-    cudaError_t e = launch_topw_select_rows(dm, P.B * P.H, n_prev * P.w, P.w, P.w_heads, P.H, sel2, P.w, s);
+    cudaError_t e = launch_topw_select_rows(dm, P.B * P.H, n_prev * P.w, P.w, P.w_heads, P.H, sel2, nullptr, P.w, s);
     if (e != cudaSuccess) return DMA_ERR_CUDA;
     const size_t smem = (size_t)L.cap * (sizeof(uint64_t) + sizeof(int32_t));
     if (ensure_smem_limit(cp_union_kernel, (int)smem) != cudaSuccess) return DMA_ERR_CUDA;

@@ -57,6 +57,7 @@ struct Plan {
   size_t off_status, off_counts, off_lists, off_sel;
   size_t off_q16, off_k16, off_v16, off_do16;  // bf16 copies of f32 Q, K, V, dO (dtype f32 only)
   size_t off_dec_part;                 // decode partials: [B*H*n_split][d + 2] f32
+  size_t off_seld;                     // decode: delta of each selected key, beside off_sel [B, H, sel_len] f32
   size_t off_rowD;                     // backward: D = rowsum(dO * O) [B, H, Nq] f32
   size_t off_olo;                      // bf16 prefill/training: O - bf16(O) as bf16, blocked
                                        // [B, H][n_blocks][d / 8][128 rows][8]; 0 if none
@@ -102,9 +103,10 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
                                 cudaStream_t s);
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s);
 // Top-min(window, N) of each of `rows` rows of N values (delta desc, index asc), ascending indices into
-// sel[row * sel_stride ..]; the row's window is w_heads[row % H] clamped to [1, w] (w when w_heads is null).
+// sel[row * sel_stride ..] and, when seld is not null, their values into seld at the same places; the
+// row's window is w_heads[row % H] clamped to [1, w] (w when w_heads is null).
 cudaError_t launch_topw_select_rows(const float* delta, int rows, int N, int w, const int32_t* w_heads, int H,
-                                    int32_t* sel, int sel_stride, cudaStream_t s);
+                                    int32_t* sel, float* seld, int sel_stride, cudaStream_t s);
 cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s);
 cudaError_t launch_selftest_wait(const Plan& P, void* ws, long long limit_cycles, cudaStream_t s);
 cudaError_t launch_gate_append(const Plan& P, const void* V, const void* Delta, const float* A, float* delta,

@@ -880,8 +880,8 @@ DMA_DEVINL void sel_find_bin(SelShared& S, uint32_t need, int nbins, int tid) {
 // w-th best key has at most kSelCand keys; those are then resolved in shared memory.  A last pass
 // writes the selected positions in ascending order.
 __global__ void __launch_bounds__(kSelThreads, 2)
-topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int N, int w_max,
-                   const int32_t* __restrict__ w_heads, int H, int sel_stride) {
+topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, float* __restrict__ seld, int N,
+                   int w_max, const int32_t* __restrict__ w_heads, int H, int sel_stride) {
   extern __shared__ __align__(16) unsigned char sel_raw[];
   SelShared& S = *reinterpret_cast<SelShared*>(sel_raw);
   const int row = blockIdx.x;
@@ -889,8 +889,12 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
   const float* drow = delta + (size_t)row * N;
   const int k = min(row_window(w_heads, row, H, w_max), N);
   int32_t* out = sel + (size_t)row * sel_stride;
+  float* outd = seld != nullptr ? seld + (size_t)row * sel_stride : nullptr;   // delta of each selected key
   if (k == N) {
-    for (int i = tid; i < N; i += kSelThreads) out[i] = i;
+    for (int i = tid; i < N; i += kSelThreads) {
+      out[i] = i;
+      if (outd) outd[i] = drow[i];
+    }
     return;
   }
   // ---- key range of the row
@@ -1004,10 +1008,12 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
   int gt_run = 0, eq_run = 0;
   for (int i0 = 0; i0 < N; i0 += kSelThreads * kSelBatch) {
     uint32_t kb[kSelBatch];
+    float dv[kSelBatch];
 #pragma unroll
     for (int u = 0; u < kSelBatch; ++u) {
       const int i = i0 + u * kSelThreads + tid;
-      kb[u] = i < N ? order_key(drow[i]) : 0u;
+      dv[u] = i < N ? drow[i] : 0.f;
+      kb[u] = order_key(dv[u]);
     }
     uint32_t mg[kSelBatch], me[kSelBatch];
 #pragma unroll
@@ -1047,7 +1053,10 @@ topw_decode_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
       const bool g = (mg[u] >> lane) & 1u, e = (me[u] >> lane) & 1u;
       if (g || (e && eb < (int)need)) {
         const int o = gb + min(eb, (int)need);
-        if (o < k) out[o] = i;
+        if (o < k) {
+          out[o] = i;
+          if (outd) outd[o] = dv[u];
+        }
       }
     }
     gt_run += (int)S.red[0][0];
@@ -1117,8 +1126,8 @@ constexpr int kAppThreads = 256;
 // key L - 1 enters iff its order key is strictly larger; it then has the largest index, so the
 // ascending list loses the worst key's entry and gains L - 1 at its end.
 __global__ void __launch_bounds__(kAppThreads)
-topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, int L, int w_max,
-                   const int32_t* __restrict__ w_heads, int H, int sel_stride) {
+topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, float* __restrict__ seld, int L,
+                   int w_max, const int32_t* __restrict__ w_heads, int H, int sel_stride) {
   __shared__ uint64_t wmin[kAppThreads / 32];
   __shared__ int pos;
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1126,8 +1135,12 @@ topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
   const int w = row_window(w_heads, row, H, w_max);
   const int kp = min(L - 1, w);
   int32_t* out = sel + (size_t)row * sel_stride;
+  float* outd = seld + (size_t)row * sel_stride;   // delta of each selected key, kept beside it
   if (kp < w) {   // every key is selected
-    for (int i = tid; i < L; i += kAppThreads) out[i] = i;
+    for (int i = tid; i < L; i += kAppThreads) {
+      out[i] = i;
+      outd[i] = drow[i];
+    }
     return;
   }
   const bool implicit = L - 1 == w;   // the previous selection is every key 0 .. L-2
@@ -1148,7 +1161,11 @@ topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
   const int jw = (int)~(uint32_t)c;
   const bool enter = order_key(drow[L - 1]) > okw;
   if (implicit) {
-    for (int i = tid; i < w; i += kAppThreads) out[i] = (!enter || i < jw) ? i : i + 1;
+    for (int i = tid; i < w; i += kAppThreads) {
+      const int j = (!enter || i < jw) ? i : i + 1;
+      out[i] = j;
+      outd[i] = drow[j];
+    }
     return;
   }
   if (!enter) return;
@@ -1161,30 +1178,38 @@ topw_append_kernel(const float* __restrict__ delta, int32_t* __restrict__ sel, i
   for (int base = (p0 / kAppThreads) * kAppThreads; base < w; base += kAppThreads) {
     const int i = base + tid;
     int v = 0;
-    if (i >= p0 && i < w) v = i + 1 < w ? out[i + 1] : L - 1;
+    float dv = 0.f;
+    if (i >= p0 && i < w) {
+      v = i + 1 < w ? out[i + 1] : L - 1;
+      dv = i + 1 < w ? outd[i + 1] : drow[L - 1];
+    }
     __syncthreads();
-    if (i >= p0 && i < w) out[i] = v;
+    if (i >= p0 && i < w) {
+      out[i] = v;
+      outd[i] = dv;
+    }
     __syncthreads();
   }
 }
 
 cudaError_t launch_topw_append(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
-  topw_append_kernel<<<P.B * P.H, kAppThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel), P.N, P.w,
-                                                       P.w_heads, P.H, P.sel_len);
+  topw_append_kernel<<<P.B * P.H, kAppThreads, 0, s>>>(delta, ws_ptr<int32_t>(ws, P.off_sel),
+                                                       ws_ptr<float>(ws, P.off_seld), P.N, P.w, P.w_heads, P.H,
+                                                       P.sel_len);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topw_select_rows(const float* delta, int rows, int N, int w, const int32_t* w_heads, int H,
-                                    int32_t* sel, int sel_stride, cudaStream_t s) {
+                                    int32_t* sel, float* seld, int sel_stride, cudaStream_t s) {
   const int smem = (int)sizeof(SelShared);
   { cudaError_t ea = ensure_smem_limit(topw_decode_kernel, smem); if (ea != cudaSuccess) return ea; }
-  topw_decode_kernel<<<rows, kSelThreads, smem, s>>>(delta, sel, N, w, w_heads, H, sel_stride);
+  topw_decode_kernel<<<rows, kSelThreads, smem, s>>>(delta, sel, seld, N, w, w_heads, H, sel_stride);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topw_decode(const Plan& P, const float* delta, void* ws, cudaStream_t s) {
   return launch_topw_select_rows(delta, P.B * P.H, P.N, P.w, P.w_heads, P.H, ws_ptr<int32_t>(ws, P.off_sel),
-                                 P.sel_len, s);
+                                 ws_ptr<float>(ws, P.off_seld), P.sel_len, s);
 }
 
 }  // namespace dma
