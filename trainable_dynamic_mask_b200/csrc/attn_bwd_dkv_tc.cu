@@ -25,12 +25,13 @@
 //               dS^T (bf16) are written back over the columns of S^T and dP^T they were read from;
 //               at the end of an item, warps 0-3 write dK (x scale) and warps 4-7 dV, and each
 //               half adds its row sums of dS^T to d delta (two f32 adds onto 0: exact in any order);
-//   warp 8      TMEM allocation; one thread issues S^T = K Q^T and dP^T = V dO^T (operands in
-//               shared memory);
-//   warp 10     one thread issues dV += P^T dO and dK += dS^T Q (A from TMEM, B read N-major).
-//               Two issuing threads on different SM sub-partitions: one thread's tcgen05.mma issue
-//               rate drops well below the tensor pipe's rate while the elementwise warps keep its
-//               sub-partition busy, and each thread's commits track only its own MMAs;
+//   warp 8      TMEM allocation; one thread issues S^T = K Q^T (operands in shared memory) and
+//               dV += P^T dO (A from TMEM, B read N-major);
+//   warp 10     one thread issues dP^T = V dO^T and dK += dS^T Q.  One thread issues a tcgen05.mma
+//               about every 60-110 cycles, slower than the tensor pipe runs these M128 N64
+//               products, so the products are split evenly over two threads on different SM
+//               sub-partitions; each thread's commits track only its own MMAs, so the barriers
+//               both feed count two arrivals;
 //   warp 9      gathers the item's K and V rows (TMA tile::gather4), double-buffered across items;
 //   warp 11     loads the Q and dO tiles of each step (TMA tiles of 64 rows), three stages.
 // TMEM: S^T buffers at columns 0 and 128, dP^T at 64 and 192 (64 columns each; step T uses buffer
@@ -80,7 +81,7 @@ struct DkSmem {
 struct DkBars {
   uint64_t kv_full[2], kv_empty[2];
   uint64_t qd_full[kDkQStages], qd_empty[kDkQStages];
-  uint64_t s_full[2], ds_full[2], mma_done[2];
+  uint64_t s_full[2], ds_full[2];
   uint64_t acc_full, acc_empty, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -274,18 +275,17 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       atomicOr(status, kErrDkAlign);
       bar.abort_flag = 1;
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2; ++i) {   // barriers both issuers feed count two arrivals
       tc::mbar_init(&bar.kv_full[i], 32);
-      tc::mbar_init(&bar.kv_empty[i], 1);
-      tc::mbar_init(&bar.s_full[i], 1);
+      tc::mbar_init(&bar.kv_empty[i], 2);
+      tc::mbar_init(&bar.s_full[i], 2);
       tc::mbar_init(&bar.ds_full[i], 256);
-      tc::mbar_init(&bar.mma_done[i], 1);
     }
     for (int i = 0; i < kDkQStages; ++i) {
       tc::mbar_init(&bar.qd_full[i], 1);
       tc::mbar_init(&bar.qd_empty[i], 2);   // both MMA issuers read the stage
     }
-    tc::mbar_init(&bar.acc_full, 1);
+    tc::mbar_init(&bar.acc_full, 2);
     tc::mbar_init(&bar.acc_empty, 256);
     tc::mbar_init(&bar.drain, 2);
     tc::fence_mbar_init();
@@ -370,61 +370,53 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         for (int m = T >= kDkQStages ? T - kDkQStages : 0; m < T; ++m)
           drain_wait(&bar.qd_full[m % kDkQStages], (m / kDkQStages) & 1);
     }
-  } else if (warp == kDkMmaWarp) {
-    // ------------------------------------------------------------ S^T and dP^T issuer (one thread)
+  } else if (warp == kDkMmaWarp || warp == kDkGradWarp) {
+    // ------------------------------------------------------------ MMA issue (lane 0 of warps 8 and 10)
+    // Warp 8 issues S^T = K Q^T and dV += P^T dO, warp 10 dP^T = V dO^T and dK += dS^T Q.  Each
+    // buffer reuse is ordered by one thread's issue order: S^T(U) (dP^T(U)) overwrites the P^T (dS^T)
+    // that the same thread's dV (dK) product of step U - 2 reads, issued after the elementwise pass
+    // of U - 2 ended (tcgen05.mma of one thread run in issue order).
     if (lane == 0) {
+      const bool sv = warp == kDkMmaWarp;
       constexpr uint32_t id_sdp = tc::idesc_bf16(128, kDkBQ, false, false);
+      constexpr uint32_t id_grad = tc::idesc_bf16(128, D, false, true);
+      const uint32_t sdp_col = sv ? kDkS : kDkDP;   // S^T / P^T or dP^T / dS^T columns of a buffer
+      const uint32_t acc_col = sv ? kDkDV : kDkDK;
+      const int a_off = sv ? S::kK : S::kV;         // A of the S^T (dP^T) product: K (V) rows
+      const int b_off = sv ? S::kQ : S::kdO;        // its B: the Q (dO) tile
+      const int g_off = sv ? S::kdO : S::kQ;        // B of the gradient product, read N-major
       int T = 0, n = 0;
       bool ok = !*abort_flag;
+      auto sdp = [&](int U, uint64_t ad) -> bool {
+        const int b = U & 1, st = U % kDkQStages;
+        if (!tc::mbar_wait(&bar.qd_full[st], (U / kDkQStages) & 1, abort_flag, status, kErrDkQ)) return false;
+        tc::fence_after();
+        const uint64_t bd = tc::sdesc(smem_u32(sm + b_off + st * S::kQT), 16, 1024);
+        DkSdpSteps<0, D / 16>::run(tmem + b * kDkBuf + sdp_col, ad, bd, id_sdp);
+        tc::commit(&bar.s_full[b]);
+        return true;
+      };
       for (int r = 0; ok && item_at(r, rec, bh); ++r, ++n) {
         const int kvb = n & 1;
         if (!(ok = tc::mbar_wait(&bar.kv_full[kvb], (n >> 1) & 1, abort_flag, status, kErrDkKV))) break;
-        const uint64_t ak = tc::sdesc(smem_u32(sm + S::kK + kvb * S::kKV), 16, 1024);
-        const uint64_t av = tc::sdesc(smem_u32(sm + S::kV + kvb * S::kKV), 16, 1024);
+        const uint64_t ad = tc::sdesc(smem_u32(sm + a_off + kvb * S::kKV), 16, 1024);
         const int steps = rec.y;
+        if (!(ok = sdp(T, ad))) break;
+        if (steps == 1) tc::commit(&bar.kv_empty[kvb]);
         for (int i = 0; i < steps; ++i) {
           const int U = T + i, b = U & 1, st = U % kDkQStages;
-          if (!(ok = tc::mbar_wait(&bar.qd_full[st], (U / kDkQStages) & 1, abort_flag, status, kErrDkQ))) break;
-          // buffer b last held step U - 2: its gradient products (the other issuer) must be done
-          if (U >= 2 && !(ok = tc::mbar_wait(&bar.mma_done[b], ((U >> 1) - 1) & 1, abort_flag, status, kErrDkDone)))
-            break;
-          tc::fence_after();
-          const uint64_t bq = tc::sdesc(smem_u32(sm + S::kQ + st * S::kQT), 16, 1024);
-          const uint64_t bdo = tc::sdesc(smem_u32(sm + S::kdO + st * S::kQT), 16, 1024);
-          DkSdpSteps<0, D / 16>::run(tmem + b * kDkBuf + kDkS, ak, bq, id_sdp);
-          DkSdpSteps<0, D / 16>::run(tmem + b * kDkBuf + kDkDP, av, bdo, id_sdp);
-          tc::commit(&bar.s_full[b]);
-          tc::commit(&bar.qd_empty[st]);
-          if (i + 1 == steps) tc::commit(&bar.kv_empty[kvb]);   // K and V of the item read for the last time
-        }
-        if (!ok) break;
-        T += steps;
-      }
-      tc::commit(&bar.drain);
-      drain_wait(&bar.drain, 0);
-    }
-    __syncwarp();
-  } else if (warp == kDkGradWarp) {
-    // ------------------------------------------------------------ dV and dK issuer (one thread)
-    if (lane == 0) {
-      constexpr uint32_t id_grad = tc::idesc_bf16(128, D, false, true);
-      int T = 0, n = 0;
-      bool ok = !*abort_flag;
-      for (int r = 0; ok && item_at(r, rec, bh); ++r, ++n) {
-        const int steps = rec.y;
-        for (int i = 0; i < steps; ++i) {
-          // dV += P^T(U) dO(U), dK += dS^T(U) Q(U); the first step of an item starts the accumulators,
-          // which the previous item's epilogue must have read
-          const int U = T + i, b = U & 1, st = U % kDkQStages;
+          if (i + 1 < steps) {
+            if (!(ok = sdp(U + 1, ad))) break;
+            if (i + 2 == steps) tc::commit(&bar.kv_empty[kvb]);   // K (V) of the item read for the last time
+          }
+          // dV (dK) += P^T (dS^T) of step U times its dO (Q) tile; the first step of an item starts
+          // the accumulator, which the previous item's epilogue must have read
           if (!(ok = tc::mbar_wait(&bar.ds_full[b], (U >> 1) & 1, abort_flag, status, kErrDkDS))) break;
           if (i == 0 && n >= 1 && !(ok = tc::mbar_wait(&bar.acc_empty, (n - 1) & 1, abort_flag, status, kErrDkAcc)))
             break;
           tc::fence_after();
-          const uint64_t bdo = tc::sdesc(smem_u32(sm + S::kdO + st * S::kQT), kDkBQ * 128, 1024);
-          const uint64_t bq = tc::sdesc(smem_u32(sm + S::kQ + st * S::kQT), kDkBQ * 128, 1024);
-          DkGradSteps<0>::run(tmem + kDkDV, tmem + b * kDkBuf + kDkS, bdo, id_grad, i == 0 ? 0u : 1u);
-          DkGradSteps<0>::run(tmem + kDkDK, tmem + b * kDkBuf + kDkDP, bq, id_grad, i == 0 ? 0u : 1u);
-          tc::commit(&bar.mma_done[b]);
+          const uint64_t gd = tc::sdesc(smem_u32(sm + g_off + st * S::kQT), kDkBQ * 128, 1024);
+          DkGradSteps<0>::run(tmem + acc_col, tmem + b * kDkBuf + sdp_col, gd, id_grad, i == 0 ? 0u : 1u);
           tc::commit(&bar.qd_empty[st]);
         }
         if (!ok) break;

@@ -6,18 +6,25 @@
 //
 // With P the masked softmax (recomputed from the forward's LSE): dP = dO V^T, D_t = sum_c dO_tc O_tc,
 // dS = P (dP - D), dQ = scale dS K.  Work item = (b, h, block of 128 query rows) over the block's
-// live-key list (full keys first) in tiles of 128 keys; persistent CTAs, heaviest blocks first.
+// live-key list (full keys first) in tiles of 96 keys; persistent CTAs, heaviest blocks first.
 //
-// Warp roles (384 threads):
-//   warps 0-3  dS: thread r owns query row r (= TMEM lane r); per tile it reads S and dP in
-//              32-column chunks, computes P = exp2(s scale log2(e) + delta_j log2(e) - LSE_t log2(e))
-//              (mask j <= t < e_j on tiles that are not all full keys), dS = P (dP - D_t), and
-//              writes dS (bf16) over the chunk's S columns; at the end of the item it writes dQ;
-//   warp 4     allocates TMEM; one thread issues S = Q K^T and dP = dO V^T (operands in shared
-//              memory) and dQ += dS K (dS from TMEM, K from shared memory read N-major);
-//   warps 5-7  gather V rows; warps 8-11 gather Q, dO and K rows (TMA tile::gather4).
-// TMEM: S buffers [0,128) and [384,512) (tile i uses buffer i % 2, so S of tile i + 1 is computed
-// while dS of tile i feeds its dQ MMA), dP [128,256), dQ [256,256+D).
+// Warp roles (512 threads):
+//   warps 0-7  dS: warp w serves query rows 32 (w % 4) .. + 31 (= its TMEM lane quarter) and key
+//              columns 48 (w / 4) .. + 47 of each tile: it reads S and dP, computes
+//              P = exp2(s scale log2(e) + delta_j log2(e) - LSE_t log2(e)) (mask j <= t < e_j on tiles
+//              that are not all full keys), dS = P (dP - D_t), and writes dS (bf16, two per column)
+//              over the first 24 of its S columns; at the end of the item it writes half of dQ's row;
+//   warp 8     allocates TMEM; its lane 0 issues S = Q K^T (operands in shared memory) and
+//              dQ += dS K (dS from TMEM, K from shared memory read N-major);
+//   warp 9     its lane 0 issues dP = dO V^T: one thread issues a tcgen05.mma about every 60-80
+//              cycles, slower than the tensor pipe runs these 96-column products, so two threads on
+//              different sub-partitions share the issue (each commit tracks its own thread's
+//              products: barriers that wait for both count two arrivals);
+//   warps 10-15 gather rows (TMA tile::gather4): Q and dO (warps 12-15), K (warps 12-14, which also
+//              stage each K tile's key metadata delta_j log2(e), j, e_j - j in shared memory beside
+//              it) and V (warps 10, 11, 15).
+// TMEM: dQ [0, D); two tile buffers, each S (96 columns) then dP (96 columns), at 128 and 320, so
+// that S and dP of tile T + 1 are computed while the dS pass of tile T runs.
 // Every wait is bounded (tc::mbar_wait); every TMEM access sits behind warp-uniform decisions.
 #include <cuda.h>
 
@@ -26,64 +33,102 @@
 namespace dma {
 namespace {
 
-constexpr int kBqThreads = 384;
-constexpr int kBqMmaWarp = 4;
-constexpr int kBqVWarp0 = 5;    // V producers: warps 5-7, row groups 11 + 11 + 10
-constexpr int kBqKWarp0 = 8;    // Q, dO, K producers: warps 8-11, row groups 8 per warp
-// setmaxnreg: launched with 168 per thread (384 x 168 = 64512); 128 x 232 + 256 x 56 = 44032.
-constexpr int kBqRegsSoftmax = 232, kBqRegsOther = 56;
-constexpr int kBqBK = 128;      // keys per tile
-constexpr int kBqStages = 2;    // K and V stages
-constexpr uint32_t kBqS0 = 0, kBqS1 = 384, kBqDP = 128, kBqDQ = 256;   // TMEM columns
+constexpr int kBqThreads = 512;
+constexpr int kBqMmaWarp = 8;    // issues S and dQ
+constexpr int kBqDpWarp = 9;     // issues dP
+constexpr int kBqVWarp0 = 10;    // V: warps 10, 11 and 15, lanes 0-7 (row groups 0-23)
+constexpr int kBqKWarp0 = 12;    // Q and dO: warps 12-15 (row groups 0-31); K: warps 12-14 (0-23)
+// setmaxnreg: launched with 128 per thread (512 x 128 = 65536); 256 x 184 + 256 x 72 = 65536.
+constexpr int kBqRegsDs = 184, kBqRegsOther = 72;
+constexpr int kBqBK = 96;        // keys per tile
+constexpr int kBqCols = 48;      // key columns per dS thread
+// K and V stages (three each: four K stages and two V stages measured slower; seven do not fit).
+constexpr int kBqKStages = 3, kBqVStages = 3;
+constexpr uint32_t kBqDQ = 0, kBqBuf0 = 128, kBqBuf1 = 320, kBqDP = 96;   // TMEM columns (dP after S)
+
+static_assert(kBqDpWarp == kBqMmaWarp + 1 && kBqVWarp0 == kBqDpWarp + 1, "warps 8 and 9 issue, the rest produce");
 
 enum : int { kErrBqQ = 0x100000, kErrBqK = 0x200000, kErrBqV = 0x400000, kErrBqS = 0x800000,
              kErrBqDS = 0x1000000, kErrBqDQ = 0x2000000, kErrBqEmpty = 0x4000000, kErrBqAlign = 0x8000000 };
 
 template <int D>
 struct BqSmem {
-  static constexpr int kTile = (D / 64) * 128 * 128;   // 128 rows: [D/64][128][128 B]
+  static constexpr int kHalves = D / 64;                 // 64-element column halves of a row
+  static constexpr int kQTile = kHalves * 128 * 128;     // 128 rows: [halves][128][128 B]
+  static constexpr int kKHalf = kBqBK * 128;             // bytes of one column half of a K or V tile
+  static constexpr int kKTile = kHalves * kKHalf;        // 96 rows: [halves][96][128 B]
   static constexpr int kQ = 0;
-  static constexpr int kdO = kTile;
-  static constexpr int kK = 2 * kTile;                  // [kBqStages]
-  static constexpr int kV = kK + kBqStages * kTile;     // [kBqStages]
-  static constexpr int kMeta = kV + kBqStages * kTile;  // [2 buffers][dl f32 | j | e - j][128]
-  static constexpr int kBars = kMeta + 2 * 3 * kBqBK * 4;
+  static constexpr int kdO = kQTile;
+  static constexpr int kK = 2 * kQTile;                  // [kBqKStages]
+  static constexpr int kV = kK + kBqKStages * kKTile;    // [kBqVStages]
+  static constexpr int kMeta = kV + kBqVStages * kKTile; // [kBqKStages][dl f32 | j | e - j][kBqBK]
+  static constexpr int kBars = kMeta + kBqKStages * 3 * kBqBK * 4;
   static constexpr int kBytes = kBars + 256;
 };
 
 struct BqBars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kBqStages], k_empty[kBqStages], v_full[kBqStages], v_empty[kBqStages];
-  uint64_t s_full, ds_full, dq_done, drain;
+  uint64_t k_full[kBqKStages], k_empty[kBqKStages], v_full[kBqVStages], v_empty[kBqVStages];
+  uint64_t s_full[2], ds_full[2], dq_done, dq_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
 
-DMA_DEVINL void bq_sync() { asm volatile("bar.sync 1, 128;\n" ::: "memory"); }
+// tcgen05.mma issued by the lane whose `leader` is non-zero (the whole warp runs the issue loop, so
+// the descriptors stay warp-uniform), A and B from shared memory, descriptors advanced by OFFA / 16
+// and OFFB / 16; ACC: accumulate into D (else overwrite it), or -1 to take `accumulate`.
+template <uint32_t OFFA, uint32_t OFFB>
+DMA_DEVINL void bq_mma_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate,
+                          uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 a, b;\n\t"
+      "add.s64 a, %1, %5;\n\t"
+      "add.s64 b, %2, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 e, %7, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(OFFA >> 4), "n"(OFFB >> 4), "r"(leader));
+}
+// The same with A from TMEM column a + ACOL and B from shared memory at descriptor + OFFB / 16.
+template <uint32_t ACOL, uint32_t OFFB>
+DMA_DEVINL void bq_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t accumulate,
+                          uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 b;\n\t.reg .b32 at;\n\t"
+      "add.s64 b, %2, %5;\n\t"
+      "add.u32 at, %1, %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 e, %7, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [at], b, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate), "n"(OFFB >> 4), "n"(ACOL), "r"(leader));
+}
 
-// 8 K steps of an M128 N128 product with both operands K-major SW128 (128-row tiles).
-template <int KK, int NK>
-struct BqSteps {
-  DMA_DEVINL static void run(uint32_t d, uint64_t da, uint64_t db, uint32_t id) {
-    mma_ss_at<(KK >> 2) * 16384 + (KK & 3) * 32>(d, da, db, id, KK > 0 ? 1u : 0u);
-    BqSteps<KK + 1, NK>::run(d, da, db, id);
+// S = A B^T over D / 16 K steps, A a 128-row tile and B a 96-row tile, both K-major SW128.
+template <int KK, int NK, int D>
+struct BqSdp {
+  DMA_DEVINL static void run(uint32_t d, uint64_t da, uint64_t db, uint32_t id, uint32_t leader) {
+    bq_mma_ss<(KK >> 2) * BqSmem<D>::kQTile / (D / 64) + (KK & 3) * 32, (KK >> 2) * BqSmem<D>::kKHalf + (KK & 3) * 32>(
+        d, da, db, id, KK > 0 ? 1u : 0u, leader);
+    BqSdp<KK + 1, NK, D>::run(d, da, db, id, leader);
   }
 };
-template <int NK>
-struct BqSteps<NK, NK> {
-  DMA_DEVINL static void run(uint32_t, uint64_t, uint64_t, uint32_t) {}
+template <int NK, int D>
+struct BqSdp<NK, NK, D> {
+  DMA_DEVINL static void run(uint32_t, uint64_t, uint64_t, uint32_t, uint32_t) {}
 };
-// dQ (+)= dS K: 8 K steps of 16 keys, A = dS from TMEM, B = K tile read N-major.
-template <int KK, int NK>
-struct BqDqSteps {
-  DMA_DEVINL static void run(uint32_t d, uint32_t a, uint64_t db, uint32_t id, uint32_t acc0) {
-    mma_ts_at<KK>(d, a, db, id, KK > 0 ? 1u : acc0);
-    BqDqSteps<KK + 1, NK>::run(d, a, db, id, acc0);
+// dQ (+)= dS K over 6 K steps of 16 keys: keys 0-47 of dS sit in columns 0-23 of the S buffer and
+// keys 48-95 in columns 48-71 (each dS thread writes over the S columns it has read); K is read
+// N-major, 16 rows (2048 B) per step.
+template <int KK>
+struct BqDq {
+  DMA_DEVINL static void run(uint32_t d, uint32_t a, uint64_t db, uint32_t id, uint32_t acc0, uint32_t leader) {
+    bq_mma_ts<KK * 8 + (KK >= 3 ? 24 : 0), KK * 2048>(d, a, db, id, KK > 0 ? 1u : acc0, leader);
+    BqDq<KK + 1>::run(d, a, db, id, acc0, leader);
   }
 };
-template <int NK>
-struct BqDqSteps<NK, NK> {
-  DMA_DEVINL static void run(uint32_t, uint32_t, uint64_t, uint32_t, uint32_t) {}
+template <>
+struct BqDq<kBqBK / 16> {
+  DMA_DEVINL static void run(uint32_t, uint32_t, uint64_t, uint32_t, uint32_t, uint32_t) {}
 };
 
 DMA_DEVINL int bq_item_index(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
@@ -111,17 +156,22 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       bar.abort_flag = 1;
     }
     tc::mbar_init(&bar.q_full, 32);
-    tc::mbar_init(&bar.q_empty, 1);
-    for (int i = 0; i < kBqStages; ++i) {
-      tc::mbar_init(&bar.k_full[i], 32);
+    tc::mbar_init(&bar.q_empty, 2);
+    for (int i = 0; i < kBqKStages; ++i) {
+      tc::mbar_init(&bar.k_full[i], kBqBK / 4);
       tc::mbar_init(&bar.k_empty[i], 1);
-      tc::mbar_init(&bar.v_full[i], 32);
+    }
+    for (int i = 0; i < kBqVStages; ++i) {
+      tc::mbar_init(&bar.v_full[i], kBqBK / 4);
       tc::mbar_init(&bar.v_empty[i], 1);
     }
-    tc::mbar_init(&bar.s_full, 1);
-    tc::mbar_init(&bar.ds_full, 128);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bar.s_full[i], 2);
+      tc::mbar_init(&bar.ds_full[i], 8);
+    }
     tc::mbar_init(&bar.dq_done, 1);
-    tc::mbar_init(&bar.drain, 1);
+    tc::mbar_init(&bar.dq_free, 8);
+    tc::mbar_init(&bar.drain, 2);
     tc::fence_mbar_init();
   }
   if (warp == kBqMmaWarp) {
@@ -136,24 +186,23 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
 
   if (warp >= kBqMmaWarp) {
     regs_dec<kBqRegsOther>();
-    if (warp > kBqMmaWarp) {
+    if (warp >= kBqVWarp0) {
       // ---------------------------------------------------------- producers (TMA gather4)
-      const bool kside = warp >= kBqKWarp0;
-      int grp, ngrp;
-      if (kside) {
-        grp = (warp - kBqKWarp0) * 8 + lane;
-        ngrp = 8;
-      } else {
-        const int vw = warp - kBqVWarp0;
-        grp = vw * 11 + lane;
-        ngrp = vw < 2 ? 11 : 10;
-      }
-      const bool issuer = lane < ngrp;
-      const uint32_t goff = (uint32_t)(4 * grp) * 128;
+      // A warp issues TMA requests one lane after another (about one per 64-72 cycles), so the
+      // requests are spread over all six warps: Q and dO rows (32 groups of 4) over warps 12-15, K
+      // rows (24 groups) over warps 12-14 and V rows (24 groups) over warps 10, 11 and 15, lanes 0-7.
+      const bool q_role = warp >= kBqKWarp0;
+      const bool kside = q_role && warp < kBqKWarp0 + 3;
+      const int qgrp = (warp - kBqKWarp0) * 8 + lane;
+      const int grp = kside ? qgrp : (q_role ? 16 : (warp - kBqVWarp0) * 8) + lane;
+      const bool q_issuer = q_role && lane < 8;          // 32 groups of 4 query rows
+      const bool t_issuer = lane < 8;                    // 24 groups of 4 key rows
       uint64_t* full = kside ? bar.k_full : bar.v_full;
       uint64_t* empty = kside ? bar.k_empty : bar.v_empty;
       const CUtensorMap* map = kside ? &kmap : &vmap;
       const int tile_base = kside ? S::kK : S::kV;
+      const int n_st = kside ? kBqKStages : kBqVStages;
+      float* meta0 = reinterpret_cast<float*>(sm + S::kMeta);
       int tcount = 0, n_done = 0;
       bool ok = !*abort_flag;
       for (int r = 0; ok; ++r) {
@@ -167,79 +216,122 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         const int b = bh / H, h = bh % H, g = h / G, Hkv = H / G;
         const int kvrow0 = (b * Hkv + g) * N;
         const int32_t* list = lists + ((size_t)bh * n_blocks + kb) * list_cap;
-        if (kside) {
+        const float* drow = delta + (size_t)bh * N;
+        const int32_t* erow = evict + (size_t)bh * N;
+        if (q_role) {
           if (n_done > 0 && !wait_all(&bar.q_empty, (n_done - 1) & 1, abort_flag, status, kErrBqEmpty)) {
             ok = false;
             break;
           }
-          if (issuer) {   // Q and dO rows (rows past N repeat row N-1; their outputs are dropped)
+          if (q_issuer) {   // Q and dO rows (rows past N repeat row N-1; their outputs are dropped)
             int rr[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) rr[u] = bh * N + min(t0 + 4 * grp + u, N - 1);
+            for (int u = 0; u < 4; ++u) rr[u] = bh * N + min(t0 + 4 * qgrp + u, N - 1);
             mbar_arrive_expect_tx(&bar.q_full, 8 * kRowBytes);
 #pragma unroll
             for (int hf = 0; hf < D / 64; ++hf) {
-              tma_gather4(smem_u32(sm + S::kQ) + hf * 16384 + goff, &qmap, hf * 64, rr[0], rr[1], rr[2], rr[3],
-                          &bar.q_full);
-              tma_gather4(smem_u32(sm + S::kdO) + hf * 16384 + goff, &domap, hf * 64, rr[0], rr[1], rr[2], rr[3],
-                          &bar.q_full);
+              tma_gather4(smem_u32(sm + S::kQ) + hf * 128 * 128 + qgrp * 512, &qmap, hf * 64, rr[0], rr[1], rr[2],
+                          rr[3], &bar.q_full);
+              tma_gather4(smem_u32(sm + S::kdO) + hf * 128 * 128 + qgrp * 512, &domap, hf * 64, rr[0], rr[1], rr[2],
+                          rr[3], &bar.q_full);
             }
           }
         }
+        // Loads run ahead of their use so that no lane waits on one: the list entries two tiles
+        // ahead, the delta and eviction values of the keys one tile ahead (K side).
+        auto entries = [&](int i, int (&j)[4]) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int li = i * kBqBK + 4 * grp + u;
+            j[u] = t_issuer && li < n_live ? list[li] : -1;
+          }
+        };
+        auto key_values = [&](const int (&j)[4], float (&dv)[4], int (&lv)[4]) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            dv[u] = kside && j[u] >= 0 ? drow[j[u]] : 0.f;
+            lv[u] = kside && j[u] >= 0 ? erow[j[u]] : 0;
+          }
+        };
+        int jj[4], jn[4], jnn[4], lc[4], ln[4];
+        float dc[4], dn[4];
+        entries(0, jj);
+        entries(1, jn);
+        key_values(jj, dc, lc);
         for (int i = 0; i < n_tiles; ++i, ++tcount) {
-          const int st = tcount % kBqStages;
-          if (tcount >= kBqStages &&
-              !wait_all(&empty[st], ((tcount / kBqStages) - 1) & 1, abort_flag, status, kErrBqEmpty)) {
+          const int st = tcount % n_st;
+          entries(i + 2, jnn);
+          key_values(jn, dn, ln);
+          if (tcount >= n_st && !wait_all(&empty[st], ((tcount / n_st) - 1) & 1, abort_flag, status, kErrBqEmpty)) {
             ok = false;
             break;
           }
-          if (issuer) {
-            // entries past n_live are unspecified: fetch row 0 of the head there (dS is 0 for them)
-            int rr[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int li = i * kBqBK + 4 * grp + u;
-              rr[u] = kvrow0 + (li < n_live ? max(list[li], 0) : 0);
+          if (t_issuer) {
+            // entries past n_live (j = -1) fetch row 0 of the head; their dS is 0
+            const uint32_t dst = smem_u32(sm + tile_base + st * S::kKTile) + grp * 512;
+            if (kside) {
+              mbar_expect_tx(&full[st], 4 * kRowBytes);
+            } else {
+              mbar_arrive_expect_tx(&full[st], 4 * kRowBytes);
             }
-            mbar_arrive_expect_tx(&full[st], 4 * kRowBytes);
 #pragma unroll
             for (int hf = 0; hf < D / 64; ++hf)
-              tma_gather4(smem_u32(sm + tile_base + st * S::kTile) + hf * 16384 + goff, map, hf * 64, rr[0], rr[1],
-                          rr[2], rr[3], &full[st]);
+              tma_gather4(dst + hf * S::kKHalf, map, hf * 64, kvrow0 + max(jj[0], 0), kvrow0 + max(jj[1], 0),
+                          kvrow0 + max(jj[2], 0), kvrow0 + max(jj[3], 0), &full[st]);
+            if (kside) {
+              // the dS pass's per-key values, published by this lane's arrival on the K barrier
+              float* meta = meta0 + st * 3 * kBqBK;
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int row = 4 * grp + u, j = jj[u];
+                meta[row] = dc[u] * kLog2e;
+                reinterpret_cast<int32_t*>(meta)[kBqBK + row] = j;
+                reinterpret_cast<int32_t*>(meta)[2 * kBqBK + row] = j >= 0 ? lc[u] - j : 0;
+              }
+              tc::mbar_arrive(&full[st]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            jj[u] = jn[u];
+            jn[u] = jnn[u];
+            dc[u] = dn[u];
+            lc[u] = ln[u];
           }
         }
         ++n_done;
       }
-      if (!ok && issuer && tcount > 0) drain_wait(&full[(tcount - 1) % kBqStages], ((tcount - 1) / kBqStages) & 1);
-    } else if (lane == 0) {
-      // ---------------------------------------------------------- MMA issuer (warp 4, one thread)
+      if (!ok && t_issuer && tcount > 0) drain_wait(&full[(tcount - 1) % n_st], ((tcount - 1) / n_st) & 1);
+    } else {
+      // ---------------------------------------------------------- MMA issue (warps 8 and 9, lane 0)
       constexpr uint32_t idss = tc::idesc_bf16(128, kBqBK, false, false);
       constexpr uint32_t iddq = tc::idesc_bf16(128, D, false, true);
-      const uint64_t dq0 = tc::sdesc(smem_u32(sm + S::kQ), 16, 1024);
-      const uint64_t ddo0 = tc::sdesc(smem_u32(sm + S::kdO), 16, 1024);
-      const uint64_t dk0 = tc::sdesc(smem_u32(sm + S::kK), 16, 1024);
-      const uint64_t dv0 = tc::sdesc(smem_u32(sm + S::kV), 16, 1024);
-      const uint64_t dkn0 = tc::sdesc(smem_u32(sm + S::kK), 16384, 1024);   // K read N-major
+      const bool sq = warp == kBqMmaWarp;   // S and dQ (else dP)
+      const uint32_t leader = lane == 0 ? 1u : 0u;
+      const uint64_t da0 = tc::sdesc(smem_u32(sm + (sq ? S::kQ : S::kdO)), 16, 1024);
+      const uint64_t db0 = tc::sdesc(smem_u32(sm + (sq ? S::kK : S::kV)), 16, 1024);
+      const uint64_t dkn0 = tc::sdesc(smem_u32(sm + S::kK), S::kKHalf, 1024);   // K read N-major
+      auto commit = [&](uint64_t* b) {
+        if (leader) tc::commit(b);
+        __syncwarp();
+      };
       int tcount = 0, n_done = 0;
       bool ok = !*abort_flag;
-      // S(T) = Q K^T into buffer T % 2 and dP(T) = dO V^T; K and V tiles are consumed in tile order,
-      // so tile T sits in stage T % kBqStages of both
-      // dq_wait: the dQ MMA to wait for before S(T) overwrites dS(T - 2).  A parity wait is only
-      // sound on the barrier's newest or next phase, so it names the last dQ commit issued so far:
-      // T - 2 inside an item (dQ(T - 1) follows this call), T - 1 at an item's first tile.
-      auto issue_sdp = [&](int T, int dq_wait) -> bool {
-        const int ks = T % kBqStages, vs = T % kBqStages;
-        if (!tc::mbar_wait(&bar.k_full[ks], (T / kBqStages) & 1, abort_flag, status, kErrBqK)) return false;
-        if (!tc::mbar_wait(&bar.v_full[vs], (T / kBqStages) & 1, abort_flag, status, kErrBqV)) return false;
-        // the S buffer last held dS(T - 2); dP was last read by the dS pass of T - 1
-        if (dq_wait >= 0 && !tc::mbar_wait(&bar.dq_done, dq_wait & 1, abort_flag, status, kErrBqDQ)) return false;
-        if (T >= 1 && !tc::mbar_wait(&bar.ds_full, (T - 1) & 1, abort_flag, status, kErrBqDS)) return false;
+      // S(T) (warp 8) or dP(T) (warp 9) into buffer T % 2.  The buffer last held tile T - 2.  S: its
+      // dS pass ended before warp 8 issued dQ(T - 2) (which waited for it), and dQ(T - 2) reads dS
+      // there before S(T) writes it (one thread's tcgen05.mma run in issue order).  dP: warp 9 waits
+      // for the dS pass of T - 2 itself.
+      auto issue = [&](int T) -> bool {
+        const int n_st = sq ? kBqKStages : kBqVStages, st = T % n_st;
+        uint64_t* full = sq ? bar.k_full : bar.v_full;
+        if (!wait_all(&full[st], (T / n_st) & 1, abort_flag, status, sq ? kErrBqK : kErrBqV)) return false;
+        if (!sq && T >= 2 && !wait_all(&bar.ds_full[T & 1], ((T - 2) >> 1) & 1, abort_flag, status, kErrBqDS))
+          return false;
         tc::fence_after();
-        const uint32_t sbuf = tmem + ((T & 1) ? kBqS1 : kBqS0);
-        BqSteps<0, D / 16>::run(sbuf, dq0, dk0 + (uint64_t)((ks * S::kTile) >> 4), idss);
-        BqSteps<0, D / 16>::run(tmem + kBqDP, ddo0, dv0 + (uint64_t)((vs * S::kTile) >> 4), idss);
-        tc::commit(&bar.s_full);
-        tc::commit(&bar.v_empty[vs]);
+        const uint32_t dst = tmem + ((T & 1) ? kBqBuf1 : kBqBuf0) + (sq ? 0u : kBqDP);
+        BqSdp<0, D / 16, D>::run(dst, da0, db0 + (uint64_t)((st * S::kKTile) >> 4), idss, leader);
+        commit(&bar.s_full[T & 1]);
+        if (!sq) commit(&bar.v_empty[st]);
         return true;
       };
       for (int r = 0; ok; ++r) {
@@ -249,41 +341,53 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         const int n_live = counts[((size_t)bh * n_blocks + kb) * 2 + 1];
         const int n_tiles = (n_live + kBqBK - 1) / kBqBK;
         if (n_tiles == 0) continue;
-        if (!(ok = tc::mbar_wait(&bar.q_full, n_done & 1, abort_flag, status, kErrBqQ))) break;
+        if (!(ok = wait_all(&bar.q_full, n_done & 1, abort_flag, status, kErrBqQ))) break;
         tc::fence_after();
-        if (!(ok = issue_sdp(tcount, tcount - 1))) break;
-        if (n_tiles == 1) tc::commit(&bar.q_empty);
+        if (!sq) {
+          for (int i = 0; i < n_tiles && ok; ++i) ok = issue(tcount + i);
+          if (!ok) break;
+          commit(&bar.q_empty);   // dO read for the last time
+          tcount += n_tiles;
+          ++n_done;
+          continue;
+        }
+        if (!(ok = issue(tcount))) break;
+        if (n_tiles == 1) commit(&bar.q_empty);
         for (int i = 0; i < n_tiles && ok; ++i) {
           const int T = tcount + i;
-          if (!(ok = tc::mbar_wait(&bar.ds_full, T & 1, abort_flag, status, kErrBqDS))) break;
           if (i + 1 < n_tiles) {
-            if (!(ok = issue_sdp(T + 1, T - 1))) break;
-            if (i + 2 == n_tiles) tc::commit(&bar.q_empty);   // Q and dO read for the last time
+            if (!(ok = issue(T + 1))) break;
+            if (i + 2 == n_tiles) commit(&bar.q_empty);   // Q read for the last time
           }
-          // dQ (+)= dS(T) K(T); then K(T)'s stage is free
+          if (!(ok = wait_all(&bar.ds_full[T & 1], (T >> 1) & 1, abort_flag, status, kErrBqDS))) break;
+          // the first dQ product of an item overwrites the accumulator the last item's rows were read from
+          if (i == 0 && n_done > 0 &&
+              !(ok = wait_all(&bar.dq_free, (n_done - 1) & 1, abort_flag, status, kErrBqDQ)))
+            break;
           tc::fence_after();
-          const int ks = T % kBqStages;
-          const uint32_t sbuf = tmem + ((T & 1) ? kBqS1 : kBqS0);
-          BqDqSteps<0, kBqBK / 16>::run(tmem + kBqDQ, sbuf, dkn0 + (uint64_t)((ks * S::kTile) >> 4), iddq,
-                                        i == 0 ? 0u : 1u);
-          tc::commit(&bar.dq_done);
-          tc::commit(&bar.k_empty[ks]);
+          const int st = T % kBqKStages;
+          BqDq<0>::run(tmem + kBqDQ, tmem + ((T & 1) ? kBqBuf1 : kBqBuf0), dkn0 + (uint64_t)((st * S::kKTile) >> 4),
+                       iddq, i == 0 ? 0u : 1u, leader);
+          commit(&bar.k_empty[st]);
+          if (i + 1 == n_tiles) commit(&bar.dq_done);
         }
         tcount += n_tiles;
         ++n_done;
       }
-      tc::commit(&bar.drain);
-      drain_wait(&bar.drain, 0);
+      commit(&bar.drain);
+      if (leader) drain_wait(&bar.drain, 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ dS and dQ rows (warps 0-3)
-    regs_inc<kBqRegsSoftmax>();
-    const int r = tid;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float* meta = reinterpret_cast<float*>(sm + S::kMeta);   // [2 buffers][dl | j | len][128]
+    // ------------------------------------------------------------ dS and dQ rows (warps 0-7)
+    regs_inc<kBqRegsDs>();
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;                       // query row of the block = TMEM lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int c0 = half * kBqCols;                           // this thread's key columns [c0, c0 + 48)
+    const float* meta0 = reinterpret_cast<const float*>(sm + S::kMeta);
     const uint64_t sc2 = f2(scale_log2, scale_log2);
-    int tcount = 0;
+    int tcount = 0, n_done = 0;
     bool ok = !*abort_flag;
     for (int rr = 0; ok; ++rr) {
       const int q = bq_item_index(rr, cta, n_ctas);
@@ -299,88 +403,70 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
       const float lse2 = valid ? LSE[(size_t)bh * N + t] * kLog2e : INFINITY;
       const float Dt = valid ? Drow[(size_t)bh * N + t] : 0.f;
       const uint64_t nl2 = f2(-lse2, -lse2), nD2 = f2(-Dt, -Dt);
-      const int32_t* list = lists + ((size_t)bh * n_blocks + kb) * list_cap;
-      const float* drow = delta + (size_t)bh * N;
-      const int32_t* erow = evict + (size_t)bh * N;
-      // this thread's entry of tile i: j (list), then delta_j and e_j - j; entries past n_live masked
-      auto entry_j = [&](int i) { const int li = i * kBqBK + r; return li < n_live ? list[li] : -1; };
-      int j_c = entry_j(0), j_n = n_tiles > 1 ? entry_j(1) : -1;
-      float dl_c = j_c >= 0 ? drow[j_c] * kLog2e : 0.f;
-      int ln_c = j_c >= 0 ? erow[j_c] - j_c : 0;
       for (int i = 0; i < n_tiles; ++i) {
-        const int T = tcount + i;
-        // next tile's metadata loads (independent of this tile's work)
-        const int j_nn = i + 2 < n_tiles ? entry_j(i + 2) : -1;
-        const float dl_n = j_n >= 0 ? drow[j_n] * kLog2e : 0.f;
-        const int ln_n = j_n >= 0 ? erow[j_n] - j_n : 0;
-        float* buf = meta + (T & 1) * 3 * kBqBK;   // by the CTA's tile count: alternates across items too
-        buf[r] = dl_c;
-        reinterpret_cast<int32_t*>(buf)[kBqBK + r] = j_c;
-        reinterpret_cast<int32_t*>(buf)[2 * kBqBK + r] = ln_c;
-        if (!wait_all(&bar.s_full, T & 1, abort_flag, status, kErrBqS)) {
+        const int T = tcount + i, st = T % kBqKStages;
+        if (!wait_all(&bar.s_full[T & 1], (T >> 1) & 1, abort_flag, status, kErrBqS) ||
+            !wait_all(&bar.k_full[st], (T / kBqKStages) & 1, abort_flag, status, kErrBqK)) {
           ok = false;
           break;
         }
         tc::fence_after();
-        bq_sync();
-        const uint32_t sbuf = tmem + ((T & 1) ? kBqS1 : kBqS0) + lane_base;
-        const uint32_t dpb = tmem + kBqDP + lane_base;
+        const uint32_t sb = tmem + ((T & 1) ? kBqBuf1 : kBqBuf0) + lane_base + c0;
+        uint32_t sa[32], sbv[16], pa[32], pb[16];
+        tc::tmem_ld32(sb, sa);
+        tc::tmem_ld16(sb + 32, sbv);
+        tc::tmem_ld32(sb + kBqDP, pa);
+        tc::tmem_ld16(sb + kBqDP + 32, pb);
+        const float* meta = meta0 + st * 3 * kBqBK;
+        const float2* dl2 = reinterpret_cast<const float2*>(meta) + c0 / 2;
+        const int2* jj2 = reinterpret_cast<const int2*>(meta + kBqBK) + c0 / 2;
+        const int2* ln2 = reinterpret_cast<const int2*>(meta + 2 * kBqBK) + c0 / 2;
         const bool full_tile = (i + 1) * kBqBK <= n_full;
-        const float2* dl2 = reinterpret_cast<const float2*>(buf);
-        const int2* jj2 = reinterpret_cast<const int2*>(buf + kBqBK);
-        const int2* ln2 = reinterpret_cast<const int2*>(buf + 2 * kBqBK);
-#pragma unroll
-        for (int c = 0; c < kBqBK / 32; ++c) {
-          uint32_t sv[32], pv[32], pk[16];
-          tc::tmem_ld32(sbuf + c * 32, sv);
-          tc::tmem_ld32(dpb + c * 32, pv);
-          tc::tmem_wait_ld();
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int k = c * 32 + 2 * u;
-            const float2 d = dl2[k / 2];
-            // x = s scale log2(e) + delta_j log2(e) - LSE_t log2(e)
-            const uint64_t x2 = f2_add(
-                f2_fma(f2(__uint_as_float(sv[2 * u]), __uint_as_float(sv[2 * u + 1])), sc2, f2(d.x, d.y)), nl2);
-            float x0, x1;
-            f2_split(x2, x0, x1);
-            float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            if (!full_tile) {
-              const int2 jv = jj2[k / 2], lv = ln2[k / 2];
-              p0 = (uint32_t)(t - jv.x) < (uint32_t)lv.x ? p0 : 0.f;
-              p1 = (uint32_t)(t - jv.y) < (uint32_t)lv.y ? p1 : 0.f;
-            }
-            // dS = P (dP - D_t)
-            const uint64_t ds2 =
-                f2_mul(f2(p0, p1), f2_add(f2(__uint_as_float(pv[2 * u]), __uint_as_float(pv[2 * u + 1])), nD2));
-            float ds0, ds1;
-            f2_split(ds2, ds0, ds1);
-            pk[u] = pack_bf16x2(ds0, ds1);
+        // dS of key columns c0 + 2u and c0 + 2u + 1, packed
+        auto ds_pair = [&](int u, uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1) -> uint32_t {
+          const float2 d = dl2[u];
+          // x = s scale log2(e) + delta_j log2(e) - LSE_t log2(e)
+          const uint64_t x2 = f2_add(f2_fma(f2(__uint_as_float(s0), __uint_as_float(s1)), sc2, f2(d.x, d.y)), nl2);
+          float x0, x1;
+          f2_split(x2, x0, x1);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (!full_tile) {
+            const int2 jv = jj2[u], lv = ln2[u];
+            p0 = (uint32_t)(t - jv.x) < (uint32_t)lv.x ? p0 : 0.f;
+            p1 = (uint32_t)(t - jv.y) < (uint32_t)lv.y ? p1 : 0.f;
           }
-          // dS of columns [32c, 32c + 32) goes to S columns [16c, 16c + 16), already read
-          tc::tmem_st16(sbuf + c * 16, pk);
-        }
+          // dS = P (dP - D_t)
+          const uint64_t ds2 = f2_mul(f2(p0, p1), f2_add(f2(__uint_as_float(d0), __uint_as_float(d1)), nD2));
+          float ds0, ds1;
+          f2_split(ds2, ds0, ds1);
+          return pack_bf16x2(ds0, ds1);
+        };
+        uint32_t lo[16], hi[8];
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 16; ++u) lo[u] = ds_pair(u, sa[2 * u], sa[2 * u + 1], pa[2 * u], pa[2 * u + 1]);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) hi[u] = ds_pair(16 + u, sbv[2 * u], sbv[2 * u + 1], pb[2 * u], pb[2 * u + 1]);
+        // dS of columns [c0, c0 + 48) goes to S columns [c0, c0 + 24), already read by this thread
+        tc::tmem_st16(sb, lo);
+        tc::tmem_st8(sb + 16, hi);
         tc::tmem_wait_st();
         tc::fence_before();
-        tc::mbar_arrive(&bar.ds_full);
-        j_c = j_n;
-        j_n = j_nn;
-        dl_c = dl_n;
-        ln_c = ln_n;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bar.ds_full[T & 1]);
       }
       if (!ok) break;
-      // ---- dQ row = scale * dQ_acc, after the item's last dQ MMA
-      const int last = tcount + n_tiles - 1;
-      if (!wait_all(&bar.dq_done, last & 1, abort_flag, status, kErrBqDQ)) {
+      // ---- dQ row = scale * dQ_acc (this warp's half of the columns), after the item's last dQ MMA
+      if (!wait_all(&bar.dq_done, n_done & 1, abort_flag, status, kErrBqDQ)) {
         ok = false;
         break;
       }
       tc::fence_after();
-      OutT* orow = dQ + ((size_t)bh * N + (valid ? t : 0)) * D;
+      OutT* orow = dQ + ((size_t)bh * N + (valid ? t : 0)) * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t ov[32];
-        tc::tmem_ld32(tmem + kBqDQ + lane_base + c * 32, ov);
+        tc::tmem_ld32(tmem + kBqDQ + lane_base + half * (D / 2) + c * 32, ov);
         tc::tmem_wait_ld();
         float of[32];
 #pragma unroll
@@ -388,7 +474,10 @@ bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant
         if (valid) store_row32(orow + c * 32, of);
       }
       tc::fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bar.dq_free);
       tcount += n_tiles;
+      ++n_done;
     }
   }
   tc::fence_before();

@@ -16,6 +16,12 @@ DMA_DEVINL void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
                : "memory");
 }
 
+// Raises the barrier's expected transaction bytes without arriving (the arrival comes later).
+DMA_DEVINL void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
 // Four rows (r0..r3) x 64 columns starting at column `col` of a 2-D tensor map, written as four
 // consecutive 128-byte rows at `dst` (the map's 128-byte swizzle applies); completion is counted
 // in bytes on `bar`.
@@ -46,7 +52,7 @@ DMA_DEVINL bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort_fla
 // Wait that ignores the abort flag, for draining copies in flight after an abort (bounded).
 DMA_DEVINL void drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
-  while (!tc::mbar_try_wait(bar, parity) && clock64() - t0 < 200000000LL) {
+  while (!tc::mbar_try_wait_sleep(bar, parity, 20000u) && clock64() - t0 < 200000000LL) {
   }
 }
 
