@@ -73,8 +73,8 @@ struct DkSmem {
   static constexpr int kV = 2 * kKV;                    // [2]
   static constexpr int kQ = 4 * kKV;                    // [kDkQStages]
   static constexpr int kdO = kQ + kDkQStages * kQT;     // [kDkQStages]
-  static constexpr int kMeta = kdO + kDkQStages * kQT;  // [8 warps][32 columns] float2 (lse2, D)
-  static constexpr int kBars = kMeta + 8 * 32 * 8;
+  static constexpr int kMeta = kdO + kDkQStages * kQT;  // [kDkQStages][64 columns] float2 (lse2, D)
+  static constexpr int kBars = kMeta + kDkQStages * kDkBQ * 8;
   static constexpr int kBytes = kBars + 256;
 };
 
@@ -279,14 +279,14 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       tc::mbar_init(&bar.kv_full[i], 32);
       tc::mbar_init(&bar.kv_empty[i], 2);
       tc::mbar_init(&bar.s_full[i], 2);
-      tc::mbar_init(&bar.ds_full[i], 256);
+      tc::mbar_init(&bar.ds_full[i], 8);   // one arrival per elementwise warp
     }
     for (int i = 0; i < kDkQStages; ++i) {
-      tc::mbar_init(&bar.qd_full[i], 1);
+      tc::mbar_init(&bar.qd_full[i], 32);   // the loader warp's lanes
       tc::mbar_init(&bar.qd_empty[i], 2);   // both MMA issuers read the stage
     }
     tc::mbar_init(&bar.acc_full, 2);
-    tc::mbar_init(&bar.acc_empty, 256);
+    tc::mbar_init(&bar.acc_empty, 8);
     tc::mbar_init(&bar.drain, 2);
     tc::fence_mbar_init();
   }
@@ -343,21 +343,37 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       for (int m = n >= 2 ? n - 2 : 0; m < n; ++m) drain_wait(&bar.kv_full[m & 1], (m >> 1) & 1);
   } else if (warp == kDkQWarp) {
     // ------------------------------------------------------------ Q and dO tiles of each step
-    if (lane == 0) {
-      int T = 0;
-      bool ok = !*abort_flag;
-      for (int r = 0; ok && item_at(r, rec, bh); ++r) {
-        for (int i = 0; i < rec.y; ++i, ++T) {
-          const int st = T % kDkQStages;
-          if (T >= kDkQStages &&
-              !tc::mbar_wait(&bar.qd_empty[st], ((T / kDkQStages) - 1) & 1, abort_flag, status, kErrDkEmpty)) {
-            ok = false;
-            break;
-          }
+    // Lane 0 loads the tiles; every lane also stages (LSE_t log2 e, D_t) of two of the step's 64
+    // query columns in shared memory beside them (published by its arrival on the stage's barrier;
+    // the values are loaded a step ahead, so no lane waits on a load).  Columns past N get
+    // (+inf, 0): P = 0 there.
+    int T = 0;
+    bool ok = !*abort_flag;
+    float2* metaq = reinterpret_cast<float2*>(sm + S::kMeta);
+    for (int r = 0; ok && item_at(r, rec, bh); ++r) {
+      const size_t hrow = (size_t)bh * N;
+      auto load_meta = [&](int i, float4& m) {
+        const int t = rec.x + i * kDkBQ + 2 * lane;
+        m.x = t < N ? LSE[hrow + t] * kLog2e : INFINITY;
+        m.y = t < N ? Drow[hrow + t] : 0.f;
+        m.z = t + 1 < N ? LSE[hrow + t + 1] * kLog2e : INFINITY;
+        m.w = t + 1 < N ? Drow[hrow + t + 1] : 0.f;
+      };
+      float4 mc, mn;
+      load_meta(0, mc);
+      for (int i = 0; i < rec.y; ++i, ++T) {
+        const int st = T % kDkQStages;
+        if (i + 1 < rec.y) load_meta(i + 1, mn);
+        if (T >= kDkQStages &&
+            !wait_all(&bar.qd_empty[st], ((T / kDkQStages) - 1) & 1, abort_flag, status, kErrDkEmpty)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
           // rows past this head's N belong to the next head or lie past the tensor (zero fill): the
           // mask drops every pair with t >= N
           const int y = bh * N + rec.x + i * kDkBQ;
-          mbar_arrive_expect_tx(&bar.qd_full[st], 2 * kDkBQ * kRowBytes);
+          mbar_expect_tx(&bar.qd_full[st], 2 * kDkBQ * kRowBytes);
 #pragma unroll
           for (int hf = 0; hf < D / 64; ++hf) {
             tma_tile_2d(smem_u32(sm + S::kQ + st * S::kQT) + hf * (kDkBQ * 128), &qmap, hf * 64, y, &bar.qd_full[st]);
@@ -365,11 +381,14 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
                         &bar.qd_full[st]);
           }
         }
+        reinterpret_cast<float4*>(metaq + st * kDkBQ)[lane] = mc;
+        tc::mbar_arrive(&bar.qd_full[st]);
+        mc = mn;
       }
-      if (!ok)
-        for (int m = T >= kDkQStages ? T - kDkQStages : 0; m < T; ++m)
-          drain_wait(&bar.qd_full[m % kDkQStages], (m / kDkQStages) & 1);
     }
+    if (!ok && lane == 0)
+      for (int m = T >= kDkQStages ? T - kDkQStages : 0; m < T; ++m)
+        drain_wait(&bar.qd_full[m % kDkQStages], (m / kDkQStages) & 1);
   } else if (warp == kDkMmaWarp || warp == kDkGradWarp) {
     // ------------------------------------------------------------ MMA issue (lane 0 of warps 8 and 10)
     // Warp 8 issues S^T = K Q^T and dV += P^T dO, warp 10 dP^T = V dO^T and dK += dS^T Q.  Each
@@ -432,8 +451,7 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int hf = warp >> 2, qd = warp & 3;
     const int r = 32 * qd + lane;   // key row of the item = TMEM lane
     const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
-    float2* meta = reinterpret_cast<float2*>(sm + S::kMeta) + warp * 32;   // this warp's columns
-    const float4* meta4 = reinterpret_cast<const float4*>(meta);
+    const float2* metaq = reinterpret_cast<const float2*>(sm + S::kMeta);   // [stage][64 columns]
     const uint64_t sc2 = f2(scale_log2, scale_log2);
     int T = 0, n = 0;
     bool ok = !*abort_flag;
@@ -446,23 +464,16 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const int len = jr >= 0 ? e - jr : 0;
       const uint64_t dl2 = f2(dl, dl);
       float dd = 0.f;
-      // (LSE_t log2 e, D_t) of this lane's column of step i; columns past N get (+inf, 0): P = 0
-      auto load_meta = [&](int i) -> float2 {
-        const int t = rec.x + i * kDkBQ + 32 * hf + lane;
-        return t < N ? make_float2(LSE[hrow + t] * kLog2e, Drow[hrow + t]) : make_float2(INFINITY, 0.f);
-      };
-      float2 mnext = load_meta(0);
       for (int i = 0; i < steps; ++i) {
-        const int U = T + i, b = U & 1;
-        __syncwarp();
-        meta[lane] = mnext;
-        __syncwarp();
-        if (i + 1 < steps) mnext = load_meta(i + 1);
-        if (!wait_all(&bar.s_full[b], (U >> 1) & 1, abort_flag, status, kErrDkS)) {
+        const int U = T + i, b = U & 1, st = U % kDkQStages;
+        // (LSE_t log2 e, D_t) of the step's columns, staged beside its Q / dO tiles
+        if (!wait_all(&bar.s_full[b], (U >> 1) & 1, abort_flag, status, kErrDkS) ||
+            !wait_all(&bar.qd_full[st], (U / kDkQStages) & 1, abort_flag, status, kErrDkQ)) {
           ok = false;
           break;
         }
         tc::fence_after();
+        const float4* meta4 = reinterpret_cast<const float4*>(metaq + st * kDkBQ + 32 * hf);
         const uint32_t sb = tmem + b * kDkBuf + kDkS + lane_base + 32 * hf;
         const uint32_t pb = tmem + b * kDkBuf + kDkDP + lane_base + 32 * hf;
         uint32_t sv[32], pv[32], pk[16], dk[16];
@@ -497,7 +508,8 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tc::tmem_st16(pb, dk);
         tc::tmem_wait_st();
         tc::fence_before();
-        tc::mbar_arrive(&bar.ds_full[b]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bar.ds_full[b]);
       }
       if (!ok) break;
       // ---- epilogue: dK (warps 0-3) or dV (warps 4-7) rows of the item's keys, f32 partials
@@ -525,7 +537,8 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
       }
       tc::fence_before();
-      tc::mbar_arrive(&bar.acc_empty);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&bar.acc_empty);
       if (jr >= 0) atomicAdd(d_delta + hrow + jr, dd);
       T += steps;
     }
