@@ -212,12 +212,40 @@ topw_thresh_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__
 // ---------------------------------------------------------------- eviction index (per chunk)
 
 constexpr int kEvThreads = 128;
+constexpr int kEvOwnTMaxN = kEvThreads * 32;   // rows up to this length: thresholds inside the kernel
+
+// Index of the w-th (1-based) set bit of a bitmap of nw <= kEvThreads words, one word per thread;
+// every thread of the CTA calls it and gets the result.  The bitmap must hold at least w set bits.
+DMA_DEVINL int nth_bit_of_block(const uint32_t* bm, int nw, int w, int* warp_sums, int* result) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t x = tid < nw ? bm[tid] : 0u;
+  const int c = __popc(x);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < warp; ++i) before += warp_sums[i];
+  const int excl = before + incl - c;
+  if (c > 0 && excl < w && w <= excl + c) *result = 32 * tid + nth_set_bit(x, w - excl - 1);
+  __syncthreads();
+  const int r = *result;
+  __syncthreads();   // warp_sums and result are reused by the next call
+  return r;
+}
 
 // One CTA per (chunk k, row).  Chunk k = positions [t0, t1) resolves exactly the keys evicted
 // inside it: old keys (position < t0) with rank in (T_{k+1}, T_k], and its own keys with rank above
 // T_{k+1}.  For such a key of rank r, e = max(j, first t >= t0 with #{i <= t : rank_i < r} >= w);
 // the count over old positions follows from T_k: Sk - #{old candidates with rank >= r}, Sk being
 // min(t0, w).  Its own keys that survive the last boundary get e = N.
+// T_in == nullptr (rows of at most kEvOwnTMaxN keys): the CTA finds its boundaries' thresholds
+// itself, as the w-th smallest rank among positions [0, t0) and [0, t1), from a bitmap over ranks
+// (the ranks of a row are a permutation of 0 .. N-1; over the whole row the w-th smallest is w - 1).
 __global__ void __launch_bounds__(kEvThreads)
 topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ rank_in,
                   const int32_t* __restrict__ T_in, int32_t* __restrict__ evict, int32_t* __restrict__ status,
@@ -234,11 +262,33 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   const int t0 = k * kC, t1 = min(t0 + kC, N);
   const int32_t* prow = p_in + (size_t)row * N;
   const int32_t* rrow = rank_in + (size_t)row * N;
-  const int32_t* T = T_in + (size_t)row * (nch + 1);
   int32_t* erow = evict + (size_t)row * N;
-  const int Ta = T[k], Tb = T[k + 1], Tf = T[nch];
   const int Sk = min(t0, w);
   crank[tid] = tid < t1 - t0 ? rrow[t0 + tid] : INT_MAX;
+  int Ta, Tb, Tf;
+  if (T_in != nullptr) {
+    const int32_t* T = T_in + (size_t)row * (nch + 1);
+    Ta = T[k];
+    Tb = T[k + 1];
+    Tf = T[nch];
+  } else {
+    __shared__ uint32_t bm[kEvOwnTMaxN / 32];
+    __shared__ int warp_sums[kEvThreads / 32];
+    __shared__ int result;
+    const int nw = (N + 31) / 32;
+    for (int i = tid; i < nw; i += kEvThreads) bm[i] = 0u;
+    __syncthreads();
+    for (int j = tid; j < t0; j += kEvThreads) {
+      const int r = rrow[j];
+      atomicOr(&bm[r >> 5], 1u << (r & 31));
+    }
+    __syncthreads();
+    Ta = t0 <= w ? N : nth_bit_of_block(bm, nw, w, warp_sums, &result);
+    if (tid < t1 - t0) atomicOr(&bm[crank[tid] >> 5], 1u << (crank[tid] & 31));
+    __syncthreads();
+    Tb = t1 <= w ? N : nth_bit_of_block(bm, nw, w, warp_sums, &result);
+    Tf = N <= w ? N : w - 1;
+  }
   // old candidates in rank order: the ranks in (Tb, Ta] held by positions < t0; all loads of a round
   // are issued before its ballots
   int nL = 0;
@@ -1094,10 +1144,15 @@ cudaError_t launch_topw_prefill(const Plan& P, const float* delta, int32_t* evic
     default: e = launch_topw_rank<2048>(P, delta, skeys, pbuf, rbuf, s); break;
   }
   if (e != cudaSuccess) return e;
-  const int tsmem = nch * (nch + 1) * (int)sizeof(uint32_t);
-  { cudaError_t ea = ensure_smem_limit(topw_thresh_kernel, tsmem); if (ea != cudaSuccess) return ea; }
-  topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w, P.w_heads, P.H);
-  topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, Tbuf, evict,
+  // rows the streaming list kernel takes need the thresholds only here, inside the eviction kernel
+  const bool own_T = P.N <= kListStreamMaxN;
+  static_assert(kListStreamMaxN <= kEvOwnTMaxN, "the eviction kernel's rank bitmap covers those rows");
+  if (!own_T) {
+    const int tsmem = nch * (nch + 1) * (int)sizeof(uint32_t);
+    { cudaError_t ea = ensure_smem_limit(topw_thresh_kernel, tsmem); if (ea != cudaSuccess) return ea; }
+    topw_thresh_kernel<<<rows, kThThreads, tsmem, s>>>(pbuf, rbuf, Tbuf, P.N, P.w, P.w_heads, P.H);
+  }
+  topw_evict_kernel<<<dim3(nch, rows), kEvThreads, 0, s>>>(pbuf, rbuf, own_T ? nullptr : Tbuf, evict,
                                                             ws_ptr<int32_t>(ws, P.off_status), P.N, P.w,
                                                             P.w_heads, P.H);
   const int kp0 = P.q0 / kPairQ;
