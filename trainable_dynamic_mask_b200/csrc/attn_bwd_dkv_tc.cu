@@ -58,7 +58,7 @@ constexpr uint32_t kDkS = 0, kDkDP = 64, kDkBuf = 128, kDkDK = 256, kDkDV = 384;
 // Device status codes: bit 0x10000000 marks this kernel, the other bits the wait that gave up
 // (bits the other kernels use are avoided).
 enum : int { kErrDkKV = 0x10000010, kErrDkQ = 0x10000020, kErrDkS = 0x10000040, kErrDkDS = 0x10000080,
-             kErrDkDone = 0x10080000, kErrDkAcc = 0x30000000, kErrDkEmpty = 0x50000000, kErrDkAlign = 0x10000008 };
+             kErrDkAcc = 0x30000000, kErrDkEmpty = 0x50000000, kErrDkAlign = 0x10000008 };
 
 DMA_DEVINL void store4_from_f32(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 DMA_DEVINL void store4_from_f32(uint16_t* p, float4 v) {
