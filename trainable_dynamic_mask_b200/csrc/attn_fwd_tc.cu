@@ -23,7 +23,7 @@
 //              key that holds the row's maximum enters with P = 1 exactly: a stale reference (P up
 //              to 2^k) rounds the dominant weight to bf16 too, and in rows dominated by a few large
 //              value rows (scaled keys of the long workload) that rounding alone moved outputs by
-//              more than the parity tolerance.  A quarter of the exponentials run as a polynomial
+//              more than the parity tolerance.  An eighth of the exponentials run as a polynomial
 //              on the FMA pipe to offload the MUFU pipe;
 //   warp 8     allocates TMEM; one thread issues the MMAs: S_h = Q_h K^T (operands in shared
 //              memory) and O_h += P_h V (P_h from TMEM, V from shared memory);
@@ -58,7 +58,7 @@ constexpr int kKWarp0 = 12;                 // Q/K producers: warps 12-15, row g
 constexpr int kRegsSoftmax = 208, kRegsOther = 48;
 constexpr int kTcBK = 128;                  // keys per tile
 constexpr int kKStages = 2, kVStages = 2;
-constexpr int kPolyEvery = 4;               // one pair in kPolyEvery takes the polynomial exp2
+constexpr int kPolyEvery = 8;               // one pair in kPolyEvery takes the polynomial exp2
 constexpr int kSchedRing = 4;               // units published ahead by the scheduling thread
 constexpr int kSchedConsumers = 15;         // warps that read each published unit (all but the scheduler's)
 
