@@ -342,8 +342,7 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
   __shared__ uint32_t wor[kEvThreads / 32][kEvThreads / 32];
   static_assert(kEvThreads == kC, "one thread per chunk offset");
   const int nc = t1 - t0;
-  int cr = kC;   // rank of offset tid among the chunk's keys
-  if (tid < nc) {
+  if (tid < nc) {   // q = rank of offset tid among the chunk's keys
     const int my = crank[tid];
     int q = 0;
     const int4* c4 = reinterpret_cast<const int4*>(crank);
@@ -352,7 +351,6 @@ topw_evict_kernel(const int32_t* __restrict__ p_in, const int32_t* __restrict__ 
       const int4 v = c4[i];
       q += (v.x < my) + (v.y < my) + (v.z < my) + (v.w < my);
     }
-    cr = q;
     srank[q] = my;
     soff[q] = tid;
   }
