@@ -752,7 +752,7 @@ def leg_cp(args, world, torch, dma, peaks):
             "step_us_without_exchange": round(step_ms * 1e3, 2),
             "exchange_bytes_received_per_rank": R * cb, "candidate_buffer_bytes": cb,
             "exchange_us_at_measured_nvlink_770_GBps": round(R * cb / 770e9 * 1e6, 2),
-            "note": "unmeasured on more than one GPU: the runs of this build have one GPU",
+            "note": "not measured across GPUs: both ranks run on one GPU, the exchange is not timed",
             # per timed repetition: phase A 3 kernels per rank; phase B 7 on rank 0 (copy of its own rows,
             # top-w 5, attention) and 10 on rank 1 (merged selection: gather, select, union, then the same)
             "gpu_launches": (3 + 7 + 3 + 10) * n_rep}
